@@ -1,0 +1,176 @@
+"""The scheduling plan rule, restated in plain Python (test oracle; see package doc).
+
+The pages describe the knobs but give no formula for them (POD-Attention
+explainer, "How POD-Attention overlaps prefill and decode": 2 or 4 CTAs per SM,
+split-KV capped at two full waves, CTAs allocated in proportion to the batch's
+prefill:decode mix; FlashInfer POD PR "Limit kv split when prefill tokens <=
+1536": the split count accounts for co-located decode CTAs).  This module is
+the written rule that the C planner must reproduce bit for bit.  Parity of the
+plan is therefore unpinned by the pages; tests pin it by invariants.
+
+Rule
+  Validation: Hq % Hkv == 0; g = Hq/Hkv in 1..8; d in {64, 128}; page == 16;
+    1 <= num_sms <= 512; ctas_per_sm in {0 (auto = 2), 1, 2}; ratios >= 0;
+    max_waves >= 0 (0 = 2); min_chunk_pages >= 0 (0 = 16); P >= 0;
+    if P > 0: P <= prefill_kv_len <= 2^24; 0 <= B <= 65536; 1 <= L_r <= 2^24;
+    sum_r L_r <= 2^31 - 1.
+  Prefill items (one 128-row query tile of one query head each), longest first:
+    for t = T-1 .. 0 (T = ceil(P/128)), for h = 0 .. Hq-1:
+      (q0 = 128 t, h, kv_end = C + min(128 (t+1), P), partial = -1).
+  Decode split: W = num_sms * ctas_per_sm * 4 decode warps; cap = max_waves * W;
+    pages_r = ceil(L_r / 16); N = Hkv * sum pages_r; maxp = max pages_r;
+    c = max(min_chunk_pages, ceil(N / cap)); then c += 1 while c < maxp and
+    Hkv * sum ceil(pages_r / c) > cap.  Request r is cut into
+    S_r = ceil(pages_r / c) splits; split s covers pages
+    [floor(s pages_r / S_r), floor((s+1) pages_r / S_r)), i.e. tokens
+    [16 p0, min(16 p1, L_r)).
+  Decode items (r, kv_head, k0, k1, partial, 0, 0, 0): partial = running index
+    over (r, kv_head, s) of rows with S_r > 1, else -1; sorted by
+    (-pages, r, kv_head, s).
+  Merge items (r, kv_head, first_partial, S_r) for every (r, kv_head) with S_r > 1.
+  Ratio p:d of per-SM tickets (ticket t -> prefill iff t mod (p+d) < p):
+    explicit (ratio_p, ratio_d) reduced by gcd (a zero side gives 1:0 or 0:1);
+    proportional (both 0): no prefill -> 0:1; no decode -> 1:0; otherwise
+    cost_pre = 4 d sum over prefill rows of keys seen, times Hq (FLOPs);
+    cost_dec = 248 * 4 d Hkv sum_r L_r (bytes x 248, the measured B200
+    tensor-FLOP/s per HBM-byte/s); k = ctas_per_sm;
+    n_p = floor((2 k cost_pre + tot) / (2 tot)), tot = cost_pre + cost_dec,
+    clamped to [1, k-1] when k >= 2 and n_p = 1 when k = 1; (p, d) = (n_p, k - n_p)
+    reduced by gcd (k = 1 gives 1:0).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Sequence
+
+import numpy as np
+
+PAGE = 16
+BM = 128
+WARPS_PER_CTA = 4
+COST_RATIO = 248
+MAX_SMS = 512
+
+
+class PlanError(ValueError):
+    pass
+
+
+@dataclasses.dataclass
+class PlanRef:
+    prefill_items: np.ndarray   # int32 [n, 4]
+    decode_items: np.ndarray    # int32 [n, 8]
+    merge_items: np.ndarray     # int32 [n, 4]
+    ctas_per_sm: int
+    ratio_p: int
+    ratio_d: int
+    chunk_pages: int
+    num_partials: int
+
+
+def _ceil(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+def plan_ref(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
+             prefill_len: int, prefill_kv_len: int, decode_lens: Sequence[int], *,
+             page_size: int = 16, ctas_per_sm: int = 0, ratio_p: int = 0, ratio_d: int = 0,
+             max_waves: int = 0, min_chunk_pages: int = 0) -> PlanRef:
+    Hq, Hkv, d = int(num_q_heads), int(num_kv_heads), int(head_dim)
+    P, KVp = int(prefill_len), int(prefill_kv_len)
+    lens = [int(x) for x in decode_lens]
+    B = len(lens)
+    if Hq <= 0 or Hkv <= 0 or Hq % Hkv:
+        raise PlanError("invalid head counts")
+    g = Hq // Hkv
+    if g > 8 or d not in (64, 128) or page_size != PAGE:
+        raise PlanError("unsupported")
+    if not (1 <= num_sms <= MAX_SMS) or ctas_per_sm not in (0, 1, 2):
+        raise PlanError("invalid launch knobs")
+    if ratio_p < 0 or ratio_d < 0 or max_waves < 0 or min_chunk_pages < 0:
+        raise PlanError("invalid knobs")
+    if P < 0 or (P > 0 and not (P <= KVp <= (1 << 24))):
+        raise PlanError("invalid prefill lengths")
+    if B > 65536 or any(not (1 <= L <= (1 << 24)) for L in lens) or sum(lens) > (1 << 31) - 1:
+        raise PlanError("invalid decode lengths")
+    k = 2 if ctas_per_sm == 0 else ctas_per_sm
+    waves = 2 if max_waves == 0 else max_waves
+    minc = 16 if min_chunk_pages == 0 else min_chunk_pages
+    C = KVp - P if P > 0 else 0
+
+    # prefill items, longest (last) tile first
+    pre = []
+    T = _ceil(P, BM)
+    for t in range(T - 1, -1, -1):
+        for h in range(Hq):
+            pre.append((BM * t, h, C + min(BM * (t + 1), P), -1))
+
+    # decode split
+    W = num_sms * k * WARPS_PER_CTA
+    cap = waves * W
+    pages = [_ceil(L, PAGE) for L in lens]
+    N = Hkv * sum(pages)
+    maxp = max(pages) if pages else 0
+    c = max(minc, _ceil(N, cap))
+    while c < maxp and Hkv * sum(_ceil(p, c) for p in pages) > cap:
+        c += 1
+    dec = []
+    merge = []
+    npart = 0
+    for r in range(B):
+        S = _ceil(pages[r], c) if pages[r] > 0 else 1
+        for kvh in range(Hkv):
+            first = npart
+            for s in range(S):
+                p0 = (s * pages[r]) // S
+                p1 = ((s + 1) * pages[r]) // S
+                part = -1
+                if S > 1:
+                    part = npart
+                    npart += 1
+                dec.append((p1 - p0, r, kvh, s, (r, kvh, PAGE * p0, min(PAGE * p1, lens[r]), part, 0, 0, 0)))
+            if S > 1:
+                merge.append((r, kvh, first, S))
+    dec.sort(key=lambda e: (-e[0], e[1], e[2], e[3]))
+
+    # ticket ratio
+    n_pre, n_dec = len(pre), len(dec)
+    if ratio_p or ratio_d:
+        if ratio_p == 0:
+            p_, d_ = 0, 1
+        elif ratio_d == 0:
+            p_, d_ = 1, 0
+        else:
+            gg = math.gcd(ratio_p, ratio_d)
+            p_, d_ = ratio_p // gg, ratio_d // gg
+    elif n_pre == 0:
+        p_, d_ = 0, 1
+    elif n_dec == 0:
+        p_, d_ = 1, 0
+    else:
+        rows_keys = 0
+        for t in range(T):
+            q0 = BM * t
+            n = min(BM, P - q0)
+            rows_keys += n * (C + 1) + n * q0 + n * (n - 1) // 2
+        cost_pre = 4 * d * Hq * rows_keys
+        cost_dec = COST_RATIO * 4 * d * Hkv * sum(lens)
+        tot = cost_pre + cost_dec
+        n_p = (2 * k * cost_pre + tot) // (2 * tot)
+        if k >= 2:
+            n_p = min(max(n_p, 1), k - 1)
+        else:
+            n_p = 1
+        p_, d_ = n_p, k - n_p
+        if d_ == 0:
+            p_ = 1
+        else:
+            gg = math.gcd(p_, d_)
+            p_, d_ = p_ // gg, d_ // gg
+
+    def arr(rows, w):
+        a = np.asarray(rows, dtype=np.int32)
+        return a.reshape(len(rows), w)
+
+    return PlanRef(arr(pre, 4), arr([e[4] for e in dec], 8), arr(merge, 4), k, p_, d_, c, npart)
