@@ -1,0 +1,179 @@
+/*
+ * pod_attn.h -- C ABI of the fused hybrid-batch attention library (sm_100a).
+ *
+ * One hybrid batch = one prefill chunk (request 0: P new query tokens over C
+ * earlier tokens, causal) plus B single-token decode requests, all reading one
+ * paged KV cache.  The library runs both kinds of attention concurrently on the
+ * same SMs from ONE persistent kernel whose CTAs read their SM id and take an
+ * SM-local ticket that assigns them prefill or decode work, as in
+ * "POD-Attention: Unlocking Full Prefill-Decode Overlap for Faster LLM
+ * Inference" (explainer page, "How POD-Attention overlaps prefill and decode":
+ * fuse into one kernel, self-assign roles per SM, 2 threadblocks per SM,
+ * single-warp virtual decode blocks, capped KV splits, proportional allocation).
+ * Split-KV partial results are combined by a log-sum-exp merge kernel (PAT
+ * record: "the final merge performs online softmax").
+ *
+ * Math (per query head h, kv head h / (Hq/Hkv), natural-base softmax):
+ *   prefill row i (absolute position C+i): O = softmax(scale q K[0..C+i]^T) V[0..C+i]
+ *   decode request r:                      O = softmax(scale q K[0..L_r-1]^T) V[0..L_r-1]
+ * bf16 operands, fp32 accumulation and softmax, bf16 outputs.
+ *
+ * Layouts (all row-major, element type bf16 unless stated):
+ *   q_prefill   [P, Hq, d]                 o_prefill   [P, Hq, d]
+ *   q_decode    [B, Hq, d]                 o_decode    [B, Hq, d]
+ *   k_cache / v_cache  [num_blocks, Hkv, 16, d]  (one 16-token page of one kv
+ *               head is contiguous); token j of a request lives in page
+ *               block_table[row][j / 16], slot j % 16.
+ *   block_table int32 [1 + B, block_table_stride]; row 0 = the prefill request
+ *               (its kv length is C + P and its last P tokens are the chunk's own
+ *               K/V, already written), row 1 + r = decode request r.
+ *   kv_lens     int32 [1 + B] on the device: [0] = C + P, [1 + r] = L_r; the
+ *               kernel checks them against the plan.
+ *   Slots past a request's length in its last page may hold any FINITE value
+ *   (the kernel zeroes masked V rows before use; K there is masked out).
+ *
+ * Ownership: the caller owns every device buffer (q, k/v cache, block table,
+ * lengths, outputs, workspace, trace).  The library never allocates device
+ * memory.  A plan is a host object owned by the library until
+ * pod_attn_plan_destroy.
+ *
+ * Errors: every entry point returns an int status (POD_OK or a negative code);
+ * nothing aborts or throws across the ABI.  Device-side problems found while
+ * the kernel runs (block id out of range, a bounded wait that expired, lengths
+ * that disagree with the plan) are recorded as a negative code in the int32
+ * error word at byte offset pod_attn_plan_info.error_offset of the workspace;
+ * the offending access is skipped (a load reads zeros), so no fault is raised.
+ */
+#ifndef POD_ATTN_H_
+#define POD_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  POD_OK = 0,
+  POD_ERR_INVALID_ARG = -1,    /* bad sizes, lengths, null pointers, misalignment */
+  POD_ERR_UNSUPPORTED = -2,    /* head_dim not 64/128, group > 8, page size not 16 */
+  POD_ERR_WORKSPACE = -3,      /* workspace smaller than the plan needs */
+  POD_ERR_CUDA = -4,           /* a CUDA runtime call failed (see pod_attn_last_cuda_error) */
+  POD_ERR_BOUNDS = -5,         /* device: block id outside [0, num_blocks) */
+  POD_ERR_TIMEOUT = -6,        /* device: a bounded wait expired; the kernel gave up */
+  POD_ERR_PLAN_MISMATCH = -7   /* device: kv_lens disagree with the plan */
+};
+
+/* config.flags */
+#define POD_FLAG_SEQUENTIAL 1u  /* ablation: prefill kernel, then decode kernel, then merge */
+#define POD_FLAG_TRACE 2u       /* record the per-item schedule into `trace` */
+
+typedef struct pod_attn_config {
+  int32_t num_q_heads;      /* Hq */
+  int32_t num_kv_heads;     /* Hkv; Hq % Hkv == 0 and Hq / Hkv <= 8 */
+  int32_t head_dim;         /* d in {64, 128} */
+  int32_t page_size;        /* tokens per KV page; must be 16 */
+  int32_t num_sms;          /* 0 = query the current device */
+  int32_t ctas_per_sm;      /* 0 = auto (2), 1 or 2 */
+  int32_t ratio_prefill;    /* ticket ratio p:d; 0:0 = proportional rule */
+  int32_t ratio_decode;
+  int32_t max_waves;        /* split-KV cap in waves of decode warps; 0 = 2 */
+  int32_t min_chunk_pages;  /* smallest split, in pages; 0 = 16 */
+  uint32_t flags;           /* POD_FLAG_* */
+} pod_attn_config;
+
+typedef struct pod_attn_plan pod_attn_plan_t;
+
+typedef struct pod_attn_plan_info {
+  int32_t num_prefill_items;  /* (128-row query tile, query head) units */
+  int32_t num_decode_items;   /* (request, kv head, key range) units */
+  int32_t num_merge_items;    /* (request, kv head) rows with more than one split */
+  int32_t num_partials;       /* split partial results held in the workspace */
+  int32_t ctas_per_sm;
+  int32_t ratio_prefill;
+  int32_t ratio_decode;
+  int32_t chunk_pages;        /* split size chosen by the plan, in pages */
+  int32_t num_sms;
+  int32_t grid;               /* CTAs of the persistent kernel */
+  int64_t workspace_bytes;
+  int64_t error_offset;       /* byte offset of the int32 device error word */
+  int64_t prefill_flops;      /* 4 d Hq sum over chunk rows of keys seen */
+  int64_t decode_flops;       /* 4 d Hq sum_r L_r */
+  int64_t kv_bytes;           /* 4 d Hkv (C + P + sum_r L_r): K and V read once */
+  int64_t qo_bytes;           /* 4 d Hq (P + B): Q read and O written once */
+} pod_attn_plan_info;
+
+/* Build the schedule for one hybrid batch on the host (no device work).
+ * prefill_qo_len = P (0 = no prefill); prefill_kv_len = C + P (ignored if P == 0);
+ * decode_kv_lens = host array of B lengths, each >= 1.  The work items, the
+ * split-KV partition and the ticket ratio follow the rule documented in
+ * oracle/plan_ref.py (the pages fix no formula).  On success *plan_out owns a
+ * new plan and *workspace_bytes_out (nullable) receives the device workspace
+ * size that pod_attn_upload / pod_attn_run need.
+ * Errors: POD_ERR_INVALID_ARG, POD_ERR_UNSUPPORTED, POD_ERR_CUDA (num_sms == 0
+ * and no device could be queried). */
+int pod_attn_plan(const pod_attn_config* cfg, int32_t prefill_qo_len, int32_t prefill_kv_len,
+                  int32_t num_decode, const int32_t* decode_kv_lens,
+                  pod_attn_plan_t** plan_out, size_t* workspace_bytes_out);
+
+/* Copy the plan's summary into *info.  Errors: POD_ERR_INVALID_ARG (null). */
+int pod_attn_plan_get_info(const pod_attn_plan_t* plan, pod_attn_plan_info* info);
+
+/* Host copies of the work tables, for bit-exact checks; any pointer may be null.
+ *   prefill_items int32 [num_prefill_items, 4]: q0, q_head, kv_end, partial (-1)
+ *   decode_items  int32 [num_decode_items, 8]:  r, kv_head, k0, k1, partial (-1 = unsplit), 0, 0, 0
+ *   merge_items   int32 [num_merge_items, 4]:   r, kv_head, first_partial, num_splits */
+int pod_attn_plan_tables(const pod_attn_plan_t* plan, int32_t* prefill_items,
+                         int32_t* decode_items, int32_t* merge_items);
+
+/* Enqueue on `stream` (a cudaStream_t; NULL = legacy default stream) the copy
+ * of the plan's work tables into `workspace` (device, >= workspace_bytes,
+ * 256-byte aligned).  Call once per plan and workspace before pod_attn_run;
+ * the host tables may be destroyed afterwards in stream order.
+ * Errors: POD_ERR_INVALID_ARG, POD_ERR_WORKSPACE, POD_ERR_CUDA. */
+int pod_attn_upload(const pod_attn_plan_t* plan, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Enqueue one hybrid-batch attention on `stream`: reset the ticket and queue
+ * counters in the workspace, launch the persistent fused kernel (or, with
+ * POD_FLAG_SEQUENTIAL in the plan's config, the prefill-only then decode-only
+ * kernels), then the LSE merge kernel when the plan has splits.  Asynchronous.
+ * q/k/v/o pointers: device, 16-byte aligned; unused sides (P == 0 or B == 0)
+ * may be null.  num_blocks = pages in each cache pool.  trace (nullable, used
+ * with POD_FLAG_TRACE): int32 [num_prefill_items + num_decode_items, 4], zeroed
+ * by the caller; entry = {smid, cta, home role (0 prefill, 1 decode), times run}.
+ * Errors: POD_ERR_INVALID_ARG, POD_ERR_WORKSPACE, POD_ERR_CUDA (launch failed). */
+int pod_attn_run(const pod_attn_plan_t* plan,
+                 const void* q_prefill, const void* q_decode,
+                 const void* k_cache, const void* v_cache, int64_t num_blocks,
+                 const int32_t* block_table, int32_t block_table_stride,
+                 const int32_t* kv_lens, float scale,
+                 void* o_prefill, void* o_decode,
+                 void* workspace, size_t workspace_bytes,
+                 int32_t* trace, void* stream);
+
+/* Record `ev_start` / `ev_stop` (cudaEvent_t, nullable) on the stream around the
+ * main attention kernel(s) of every later pod_attn_run with this plan (the
+ * fused kernel; in sequential mode the prefill+decode kernels).  Lets a caller
+ * time the dominant kernel without the counter reset and the merge. */
+int pod_attn_plan_set_events(pod_attn_plan_t* plan, void* ev_start, void* ev_stop);
+
+/* Helpers so callers without the CUDA headers can make timing events. */
+int pod_attn_event_create(void** ev_out);
+int pod_attn_event_destroy(void* ev);
+int pod_attn_event_elapsed_ms(void* ev_start, void* ev_stop, float* ms_out);
+
+/* Release a plan (null is allowed). */
+void pod_attn_plan_destroy(pod_attn_plan_t* plan);
+
+/* Static text for a status code. */
+const char* pod_attn_status_string(int status);
+
+/* Last CUDA error code seen by the library in this thread (0 = none). */
+int pod_attn_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* POD_ATTN_H_ */

@@ -1,0 +1,891 @@
+// Fused hybrid-batch attention for B200 (sm_100a): one persistent kernel runs
+// causal chunked-prefill tiles on the tcgen05 tensor cores and paged-KV decode
+// attention on the load/store path, side by side on every SM.
+//
+// Method: "POD-Attention: Unlocking Full Prefill-Decode Overlap for Faster LLM
+// Inference" (explainer page, "How POD-Attention overlaps prefill and decode"):
+//   * one kernel holds both kinds of work ("Fuse prefill and decode attention
+//     into one kernel");
+//   * a CTA's leader reads %smid and takes a ticket from an SM-local counter;
+//     the ticket picks the CTA's role at the plan's p:d ratio ("Self-assign
+//     roles per SM in software");
+//   * decode runs in single-warp virtual blocks ("Balance shared memory and
+//     threadblock count") with small tensor-core tiles ("Shrink decode tiles");
+//   * KV is split for decode parallelism, capped by the plan ("Cap prefill
+//     splitting"), and the splits are merged by log-sum-exp (PAT record).
+// B200 re-design (prior art, not the blueprint): CTAs are persistent -- the
+// ticket fixes a CTA's home role, the CTA drains that role's queue and then
+// steals from the other, so no CTA ever waits on another.  Prefill tiles are
+// 128 x 64 tcgen05 MMAs with S and P.V accumulated in TMEM, fed by TMA with
+// 128-byte swizzle straight from the 16-token pages; decode warps stage pages
+// with TMA into a per-warp ring and use m16n8k16 MMAs with keys as rows.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "pod_plan.h"
+#include "pod_ptx.cuh"
+
+namespace pod {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a healthy wait takes microseconds
+constexpr uint32_t kTmemCols = 256;                // S (64 cols) at 0, O tile (d cols) at 128
+constexpr uint32_t kTmemS = 0;
+constexpr uint32_t kTmemO = 128;
+
+enum Mode : int32_t { kFused = 0, kPrefillOnly = 1, kDecodeOnly = 2 };
+enum Role : int32_t { kRolePrefill = 0, kRoleDecode = 1 };
+
+struct alignas(64) PodParams {
+  CUtensorMap tm_k;    // K cache viewed as 2D [num_blocks*Hkv*16 rows, d], box {64, 16}, 128B swizzle
+  CUtensorMap tm_v;    // V cache, same view
+  CUtensorMap tm_q;    // Q prefill viewed as 3D [P][Hq][d], box {64, 1, 128}, 128B swizzle
+  const __nv_bfloat16* q_dec;
+  __nv_bfloat16* o_pre;
+  __nv_bfloat16* o_dec;
+  const int32_t* block_table;
+  const int32_t* kv_lens;
+  int32_t* counters;
+  const int4* pre_items;
+  const int4* dec_items;   // two int4 per item
+  float* part_o;
+  float* part_lse;
+  int32_t* trace;
+  int32_t bt_stride;
+  int32_t kv_rows;         // num_blocks * Hkv * 16 (rows of the K/V tensor maps)
+  int32_t num_blocks;
+  int32_t n_pre, n_dec;
+  int32_t Hq, Hkv, g, P, C, B;
+  int32_t ratio_p, ratio_d;
+  int32_t mode;
+  int32_t use_tmem;
+  float scale_log2;        // softmax scale * log2(e)
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int kHalves = D / 64;                      // 128-byte swizzle atoms along d
+  static constexpr int kQBytes = kBM * D * 2;                 // 128 query rows
+  static constexpr int kKTile = kBN * D * 2;                  // 64 keys
+  static constexpr int kStage = 2 * kKTile;                   // K + V
+  static constexpr bool kPAliasK = (kBN * kBM * 2 <= kKTile); // P [128 x 64] fits in the spent K tile
+  static constexpr int kPrefillSmem = kQBytes + 2 * kStage + (kPAliasK ? 0 : kBM * kBN * 2);
+  static constexpr int kPageBytes = kPage * D * 2;            // one 16-token page of one kv head
+  static constexpr int kDecStage = 2 * kPageBytes;            // K page + V page
+  static constexpr int kNS = (kPrefillSmem / kWarpsPerCta) / kDecStage;   // decode ring depth per warp
+  static constexpr int kSmem = kPrefillSmem;
+  // + 1024 slack for 1024-byte alignment; at least 80 KB so that no more than two
+  // CTAs (2 x 256 TMEM columns) can ever share an SM
+  static constexpr int kSmemAlloc = (kSmem + 1024) > 80 * 1024 ? (kSmem + 1024) : 80 * 1024;
+};
+static_assert(Cfg<128>::kNS >= 3 && Cfg<64>::kNS >= 3, "decode ring too shallow");
+
+__device__ __forceinline__ void record_error(const PodParams& p, int code, int info) {
+  if (atomicCAS(&p.counters[kErrorWord], 0, code) == 0) atomicExch(&p.counters[kErrorInfo], info);
+}
+
+// Row of the K/V tensor maps holding page `blk`, kv head `kvh`; an
+// out-of-range block id is recorded and mapped past the end (TMA reads zeros).
+__device__ __forceinline__ int kv_row(const PodParams& p, int blk, int kvh) {
+  if (blk < 0 || blk >= p.num_blocks) {
+    record_error(p, POD_ERR_BOUNDS, blk);
+    return p.kv_rows;
+  }
+  return (blk * p.Hkv + kvh) * kPage;
+}
+
+struct PrefillState {
+  uint32_t q_phase;
+  uint32_t kv_phase[2];
+  uint32_t mma_phase;
+};
+
+// Load the 64-key tile `kb` (4 pages x d/64 halves of K and V) into stage `s`.
+template <int D>
+__device__ __forceinline__ void prefill_issue_tile(const PodParams& p, uint8_t* stage, uint64_t* bar, int kb,
+                                                   int kvh, int kv_end) {
+  using CF = Cfg<D>;
+  mbar_arrive_expect_tx(bar, CF::kStage);
+#pragma unroll
+  for (int pi = 0; pi < kBN / kPage; ++pi) {
+    const int gp = kb * (kBN / kPage) + pi;
+    int row = p.kv_rows;                       // pages past the request's end read as zeros
+    if (gp * kPage < kv_end) row = kv_row(p, __ldg(&p.block_table[gp]), kvh);
+#pragma unroll
+    for (int h = 0; h < CF::kHalves; ++h) {
+      tma_load_2d(stage + h * (kBN * 128) + pi * (kPage * 128), &p.tm_k, bar, h * 64, row);
+      tma_load_2d(stage + CF::kKTile + h * (kBN * 128) + pi * (kPage * 128), &p.tm_v, bar, h * 64, row);
+    }
+  }
+}
+
+// One prefill work item: rows q0..q0+127 of query head qh against keys
+// 0..kv_end-1 of request 0 with the bottom-right causal mask.  All 128 threads;
+// thread t owns tile row t (TMEM lane t).  Returns false if a wait expired.
+template <int D>
+__device__ bool prefill_item(const PodParams& p, int item, uint8_t* smem, uint64_t* bars, uint32_t tmem,
+                             PrefillState& st) {
+  using CF = Cfg<D>;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int4 it = __ldg(&p.pre_items[item]);
+  const int q0 = it.x, qh = it.y, kv_end = it.z;
+  const int kvh = qh / p.g;
+  const int nkb = (kv_end + kBN - 1) / kBN;
+  uint64_t* bar_q = &bars[0];
+  uint64_t* bar_kv = &bars[1];
+  uint64_t* bar_mma = &bars[3];
+  uint8_t* sQ = smem;
+  uint8_t* stage0 = smem + CF::kQBytes;
+
+  if (tid == 0) {
+    if (p.kv_lens && __ldg(&p.kv_lens[0]) < kv_end) record_error(p, POD_ERR_PLAN_MISMATCH, item);
+    mbar_arrive_expect_tx(bar_q, CF::kQBytes);
+#pragma unroll
+    for (int h = 0; h < CF::kHalves; ++h) tma_load_3d(sQ + h * (kBM * 128), &p.tm_q, bar_q, h * 64, qh, q0);
+    prefill_issue_tile<D>(p, stage0, &bar_kv[0], 0, kvh, kv_end);
+  }
+
+  const uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false, false);
+  const uint32_t idesc_o = idesc_bf16_f32(kBM, D, false, true);
+  const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
+  const int row = tid;                                   // tile row
+  const int row_limit = min(p.C + q0 + row + 1, kv_end); // keys 0..row_limit-1 are visible
+  float o[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) o[c] = 0.f;
+  float m = -INFINITY, l = 0.f;
+  bool ok = true;
+
+  for (int kb = 0; kb < nkb; ++kb) {
+    const int s = kb & 1;
+    uint8_t* sK = stage0 + s * CF::kStage;
+    uint8_t* sV = sK + CF::kKTile;
+    uint8_t* sP = CF::kPAliasK ? sK : (stage0 + 2 * CF::kStage);
+    if (tid == 0) {
+      bool w = true;
+      if (kb == 0) w = mbar_wait(bar_q, st.q_phase, kWaitLimitNs);
+      w = w && mbar_wait(&bar_kv[s], st.kv_phase[s], kWaitLimitNs);
+      if (w) {
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(ka + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024);
+          umma_bf16(tmem + kTmemS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_mma);
+        if (kb + 1 < nkb) prefill_issue_tile<D>(p, stage0 + (s ^ 1) * CF::kStage, &bar_kv[s ^ 1], kb + 1, kvh, kv_end);
+      } else {
+        record_error(p, POD_ERR_TIMEOUT, 1);
+      }
+    }
+    if (kb == 0) st.q_phase ^= 1;
+    st.kv_phase[s] ^= 1;
+
+    // ---- S tile -> online softmax -> P (bf16, K-major 128B-swizzled in smem)
+    bool w1 = mbar_wait(bar_mma, st.mma_phase, kWaitLimitNs);
+    st.mma_phase ^= 1;
+    __syncwarp();
+    tc_fence_after();
+    float sv[kBN];
+    tmem_ld32(tmem + t_lane + kTmemS, sv);
+    tmem_ld32(tmem + t_lane + kTmemS + 32, sv + 32);
+    tmem_wait_ld();
+    const int lim = row_limit - kb * kBN;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kBN; ++j) {
+      sv[j] = (j < lim) ? sv[j] * p.scale_log2 : -INFINITY;
+      mx = fmaxf(mx, sv[j]);
+    }
+    const float m_new = fmaxf(m, mx);
+    const float alpha = ex2(m - m_new);
+    float rs = 0.f;
+    uint8_t* prow = sP + row * 128;
+#pragma unroll
+    for (int c = 0; c < kBN / 8; ++c) {
+      float e[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        e[j] = ex2(sv[c * 8 + j] - m_new);
+        rs += e[j];
+      }
+      uint4 v;
+      v.x = pack_bf16(e[0], e[1]);
+      v.y = pack_bf16(e[2], e[3]);
+      v.z = pack_bf16(e[4], e[5]);
+      v.w = pack_bf16(e[6], e[7]);
+      *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v;
+    }
+    l = l * alpha + rs;
+    m = m_new;
+    // zero V rows past kv_end in the last tile (they may hold anything)
+    const int valid_keys = kv_end - kb * kBN;
+    if (valid_keys < kBN) {
+      if (!mbar_wait(&bar_kv[s], st.kv_phase[s] ^ 1, kWaitLimitNs)) w1 = false;
+      const int nz = (kBN - valid_keys) * CF::kHalves * 8;   // 16-byte chunks to clear
+      for (int i = tid; i < nz; i += 128) {
+        const int chunk = i & 7, rh = i >> 3;
+        const int key = valid_keys + rh % (kBN - valid_keys), h = rh / (kBN - valid_keys);
+        *reinterpret_cast<uint4*>(sV + h * (kBN * 128) + key * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    if (__syncthreads_or(!w1)) {
+      ok = false;
+      break;
+    }
+    // ---- O tile = P V (fresh accumulator each key tile)
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t pa = smem_u32(sP), va = smem_u32(sV);
+#pragma unroll
+      for (int kk = 0; kk < kBN / 16; ++kk) {
+        const uint64_t ad = sdesc_sw128(pa + kk * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(va + kk * (16 * 128), kBN * 128, 1024);
+        umma_bf16(tmem + kTmemO, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(bar_mma);
+    }
+    const bool w2 = mbar_wait(bar_mma, st.mma_phase, kWaitLimitNs);
+    st.mma_phase ^= 1;
+    __syncwarp();
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float ov[32];
+      tmem_ld32(tmem + t_lane + kTmemO + c * 32, ov);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) o[c * 32 + j] = o[c * 32 + j] * alpha + ov[j];
+    }
+    tc_fence_before();
+    if (__syncthreads_or(!w2)) {
+      ok = false;
+      break;
+    }
+  }
+  if (!ok) {
+    if (tid == 0) record_error(p, POD_ERR_TIMEOUT, 2);
+    return false;
+  }
+  // ---- epilogue: O / l -> bf16, one 2*D-byte row per thread
+  const int q = q0 + row;
+  if (q < p.P) {
+    const float inv = 1.f / l;
+    uint4* dst = reinterpret_cast<uint4*>(p.o_pre + ((size_t)q * p.Hq + qh) * D);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      uint4 v;
+      v.x = pack_bf16(o[c * 8 + 0] * inv, o[c * 8 + 1] * inv);
+      v.y = pack_bf16(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv);
+      v.z = pack_bf16(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv);
+      v.w = pack_bf16(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
+      dst[c] = v;
+    }
+  }
+  (void)lane;
+  return true;
+}
+
+// ------------------------------------------------------------------ decode
+// One warp = one virtual decode block.  Item (r, kvh, k0, k1): the g query
+// heads of kv head kvh of decode request r against keys k0..k1-1.
+// Per 16-token page: S^T[16 keys x 8 heads] = K_page . Q^T (m16n8k16, keys as
+// rows so only the head dimension is padded), online softmax per head across
+// lanes, P^T moved into the B-operand layout with movmatrix, then
+// O^T[d x 8] += V_page^T . P^T.  Pages arrive by TMA into a kNS-deep ring.
+template <int D>
+__device__ __forceinline__ void decode_issue_page(const PodParams& p, uint8_t* ring, uint64_t* wbars, uint32_t seq,
+                                                  int bt_row, int gpage, int kvh) {
+  using CF = Cfg<D>;
+  const int s = seq % CF::kNS;
+  uint8_t* kbuf = ring + s * CF::kDecStage;
+  uint64_t* bar = &wbars[s];
+  mbar_arrive_expect_tx(bar, CF::kDecStage);
+  const int row = kv_row(p, __ldg(&p.block_table[(size_t)bt_row * p.bt_stride + gpage]), kvh);
+#pragma unroll
+  for (int h = 0; h < CF::kHalves; ++h) {
+    tma_load_2d(kbuf + h * (kPage * 128), &p.tm_k, bar, h * 64, row);
+    tma_load_2d(kbuf + CF::kPageBytes + h * (kPage * 128), &p.tm_v, bar, h * 64, row);
+  }
+}
+
+__device__ __forceinline__ uint32_t swz(int row, int col_elem) {
+  // byte offset of (row, col) inside a [rows][64 bf16] 128-byte-swizzled atom column
+  return (uint32_t)(row * 128 + ((((col_elem >> 3) ^ row) & 7) << 4));
+}
+
+template <int D>
+__device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, uint32_t& seq,
+                            volatile int* abort_flag, int home_role) {
+  using CF = Cfg<D>;
+  const int lane = threadIdx.x & 31;
+  const int g = p.g;
+  while (true) {
+    if (*abort_flag) return false;
+    int item = 0;
+    if (lane == 0) item = atomicAdd(&p.counters[kNextDecode], 1);
+    item = __shfl_sync(0xffffffffu, item, 0);
+    if (item >= p.n_dec) return true;
+    const int4 a = __ldg(&p.dec_items[2 * item]);
+    const int4 b = __ldg(&p.dec_items[2 * item + 1]);
+    const int r = a.x, kvh = a.y, k0 = a.z, k1 = a.w, part = b.x;
+    const int p0 = k0 / kPage;
+    const int np = (k1 - k0 + kPage - 1) / kPage;
+    if (lane == 0) {
+      if (p.kv_lens && __ldg(&p.kv_lens[1 + r]) < k1) record_error(p, POD_ERR_PLAN_MISMATCH, item);
+      if (p.trace) {
+        int32_t* e = p.trace + 4 * (p.n_pre + item);
+        e[0] = (int32_t)smid();
+        e[1] = blockIdx.x;
+        e[2] = home_role;
+        atomicAdd(&e[3], 1);
+      }
+      const int pre = np < CF::kNS ? np : CF::kNS;
+      for (int j = 0; j < pre; ++j) decode_issue_page<D>(p, ring, wbars, seq + j, 1 + r, p0 + j, kvh);
+    }
+    // Q^T as the B operand: thread holds head n = lane/4, d pairs (lane%4)*2 (+8)
+    uint32_t qf[D / 16][2];
+    {
+      const int n = lane >> 2;
+      const int dc = (lane & 3) * 2;
+      if (n < g) {
+        const __nv_bfloat16* qp = p.q_dec + ((size_t)r * p.Hq + kvh * g + n) * D;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          qf[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + dc));
+          qf[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + dc));
+        }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) qf[ks][0] = qf[ks][1] = 0u;
+      }
+    }
+    float acc[D / 16][4];
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
+    const int key_lo = lane >> 2;     // S^T rows held: key_lo and key_lo + 8
+    // ldmatrix lane roles
+    const int a_row = lane & 15, a_colh = (lane >> 4) * 8;                  // K as A (non-trans)
+    const int v_key = (lane & 7) + ((lane >> 4) << 3), v_colh = ((lane >> 3) & 1) * 8;  // V^T as A (trans)
+    bool ok = true;
+    int jfail = 0;
+    for (int j = 0; j < np; ++j) {
+      const uint32_t sq = seq + j;
+      const int s = sq % CF::kNS;
+      const bool w = mbar_wait(&wbars[s], (sq / CF::kNS) & 1u, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        jfail = j;
+        break;
+      }
+      uint8_t* kbuf = ring + s * CF::kDecStage;
+      uint8_t* vbuf = kbuf + CF::kPageBytes;
+      const int valid = min(kPage, k1 - (p0 + j) * kPage);
+      if (valid < kPage) {
+        // clear V rows past the end of the request: they may hold anything
+        for (int i = lane; i < (kPage - valid) * CF::kHalves * 8; i += 32) {
+          const int chunk = i & 7, rh = i >> 3;
+          const int key = valid + rh % (kPage - valid), h = rh / (kPage - valid);
+          *reinterpret_cast<uint4*>(vbuf + h * (kPage * 128) + key * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      const uint32_t kb_u = smem_u32(kbuf), vb_u = smem_u32(vbuf);
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const int col = ks * 16 + a_colh;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(kb_u + (col >> 6) * (kPage * 128) + swz(a_row, col & 63), a0, a1, a2, a3);
+        mma_16816(c, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+      }
+      // mask, scale, online softmax per head (columns (lane%4)*2 and +1)
+      const float s0 = key_lo < valid ? c[0] * p.scale_log2 : -INFINITY;
+      const float s1 = key_lo < valid ? c[1] * p.scale_log2 : -INFINITY;
+      const float s2 = key_lo + 8 < valid ? c[2] * p.scale_log2 : -INFINITY;
+      const float s3 = key_lo + 8 < valid ? c[3] * p.scale_log2 : -INFINITY;
+      float tA = fmaxf(s0, s2), tB = fmaxf(s1, s3);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        tA = fmaxf(tA, __shfl_xor_sync(0xffffffffu, tA, o));
+        tB = fmaxf(tB, __shfl_xor_sync(0xffffffffu, tB, o));
+      }
+      const float nA = fmaxf(mA, tA), nB = fmaxf(mB, tB);
+      const float alA = ex2(mA - nA), alB = ex2(mB - nB);
+      mA = nA;
+      mB = nB;
+      const float e0 = ex2(s0 - nA), e1 = ex2(s1 - nB), e2 = ex2(s2 - nA), e3 = ex2(s3 - nB);
+      lA = lA * alA + e0 + e2;
+      lB = lB * alB + e1 + e3;
+      const uint32_t pb0 = movmatrix_t(pack_bf16(e0, e1));   // keys 0..7
+      const uint32_t pb1 = movmatrix_t(pack_bf16(e2, e3));   // keys 8..15
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int col = mt * 16 + v_colh;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(vb_u + (col >> 6) * (kPage * 128) + swz(v_key, col & 63), a0, a1, a2, a3);
+        acc[mt][0] *= alA;
+        acc[mt][1] *= alB;
+        acc[mt][2] *= alA;
+        acc[mt][3] *= alB;
+        mma_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+      }
+      __syncwarp();
+      if (lane == 0 && j + CF::kNS < np) decode_issue_page<D>(p, ring, wbars, sq + CF::kNS, 1 + r, p0 + j + CF::kNS, kvh);
+    }
+    if (!ok) {
+      // drain copies still in flight into this warp's ring before giving up
+      if (lane == 0) {
+        record_error(p, POD_ERR_TIMEOUT, 3);
+        const int jend = min(np, jfail + CF::kNS);
+        for (int j = jfail + 1; j < jend; ++j) {
+          const uint32_t sq = seq + (uint32_t)j;
+          mbar_wait(&wbars[sq % CF::kNS], (sq / CF::kNS) & 1u, kWaitLimitNs / 4);
+        }
+      }
+      *abort_flag = 1;
+      return false;
+    }
+    seq += (uint32_t)np;
+    // finalize: full row sums across the 8 lanes that share a head pair
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      lA += __shfl_xor_sync(0xffffffffu, lA, o);
+      lB += __shfl_xor_sync(0xffffffffu, lB, o);
+    }
+    const int hA = (lane & 3) * 2, hB = hA + 1;
+    const float iA = 1.f / lA, iB = 1.f / lB;
+    const int d_lo = lane >> 2;
+    if (part < 0) {
+      __nv_bfloat16* ob = p.o_dec + ((size_t)r * p.Hq + kvh * g) * D;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int dd = mt * 16 + d_lo;
+        if (hA < g) {
+          ob[hA * D + dd] = __float2bfloat16_rn(acc[mt][0] * iA);
+          ob[hA * D + dd + 8] = __float2bfloat16_rn(acc[mt][2] * iA);
+        }
+        if (hB < g) {
+          ob[hB * D + dd] = __float2bfloat16_rn(acc[mt][1] * iB);
+          ob[hB * D + dd + 8] = __float2bfloat16_rn(acc[mt][3] * iB);
+        }
+      }
+    } else {
+      float* po = p.part_o + (size_t)part * g * D;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int dd = mt * 16 + d_lo;
+        if (hA < g) {
+          po[hA * D + dd] = acc[mt][0] * iA;
+          po[hA * D + dd + 8] = acc[mt][2] * iA;
+        }
+        if (hB < g) {
+          po[hB * D + dd] = acc[mt][1] * iB;
+          po[hB * D + dd + 8] = acc[mt][3] * iB;
+        }
+      }
+      if (d_lo == 0) {
+        if (hA < g) p.part_lse[(size_t)part * g + hA] = mA + __log2f(lA);
+        if (hB < g) p.part_lse[(size_t)part * g + hB] = mB + __log2f(lB);
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------- persistent kernel
+template <int D>
+__global__ void __launch_bounds__(128, 2) pod_attn_kernel(const __grid_constant__ PodParams p) {
+  using CF = Cfg<D>;
+  extern __shared__ uint8_t dyn_smem[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bars[4 + kWarpsPerCta * CF::kNS];
+  __shared__ uint32_t tmem_holder;
+  __shared__ int sh_home, sh_item;
+  __shared__ volatile int sh_abort;
+  const int tid = threadIdx.x, warp = tid >> 5;
+
+  if (tid == 0) {
+    for (int i = 0; i < 4 + kWarpsPerCta * CF::kNS; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+    sh_abort = 0;
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    int home = p.mode == kDecodeOnly ? kRoleDecode : kRolePrefill;
+    if (p.mode == kFused) {
+      const uint32_t sm = smid();
+      const int t = atomicAdd(&p.counters[kTicketBase + (int)(sm % kMaxSms)], 1);
+      const int span = p.ratio_p + p.ratio_d;
+      home = (span > 0 && (t % span) < p.ratio_p) ? kRolePrefill : kRoleDecode;
+    }
+    sh_home = home;
+  }
+  __syncwarp();
+  if (p.use_tmem && warp == 0) {
+    tmem_alloc(&tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = p.use_tmem ? tmem_holder : 0u;
+  const int home = sh_home;
+
+  PrefillState st{0u, {0u, 0u}, 0u};
+  uint32_t seq = 0;
+  uint8_t* ring = smem + warp * CF::kNS * CF::kDecStage;
+  uint64_t* wbars = &bars[4 + warp * CF::kNS];
+
+  for (int phase = 0; phase < 2; ++phase) {
+    const int role = phase == 0 ? home : 1 - home;
+    if (p.mode == kPrefillOnly && role != kRolePrefill) continue;
+    if (p.mode == kDecodeOnly && role != kRoleDecode) continue;
+    if (role == kRolePrefill) {
+      while (true) {
+        if (tid == 0) sh_item = sh_abort ? p.n_pre : atomicAdd(&p.counters[kNextPrefill], 1);
+        __syncthreads();
+        const int item = sh_item;
+        __syncthreads();
+        if (item >= p.n_pre) break;
+        if (tid == 0 && p.trace) {
+          int32_t* e = p.trace + 4 * item;
+          e[0] = (int32_t)smid();
+          e[1] = blockIdx.x;
+          e[2] = home;
+          atomicAdd(&e[3], 1);
+        }
+        if (!prefill_item<D>(p, item, smem, bars, tmem, st)) {
+          if (tid == 0) sh_abort = 1;
+          __syncthreads();
+          break;
+        }
+      }
+    } else {
+      decode_warp<D>(p, ring, wbars, seq, &sh_abort, home);
+      __syncthreads();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (p.use_tmem && warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------- LSE merge
+struct MergeParams {
+  const int4* items;       // r, kvh, first_partial, num_splits
+  const float* part_o;     // [n_part, g, D]
+  const float* part_lse;   // [n_part, g], log2 domain
+  __nv_bfloat16* o_dec;
+  int32_t n_merge, Hq, g;
+};
+
+// One CTA per (request, kv head) row with splits: O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M).
+template <int D>
+__global__ void __launch_bounds__(128) pod_merge_kernel(const MergeParams mp) {
+  const int4 it = __ldg(&mp.items[blockIdx.x]);
+  const int r = it.x, kvh = it.y, first = it.z, S = it.w;
+  const int g = mp.g;
+  for (int idx = threadIdx.x; idx < g * D; idx += blockDim.x) {
+    const int h = idx / D, dd = idx % D;
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldg(&mp.part_lse[(size_t)(first + s) * g + h]));
+    float num = 0.f, den = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float w = ex2(__ldg(&mp.part_lse[(size_t)(first + s) * g + h]) - M);
+      num += w * __ldg(&mp.part_o[((size_t)(first + s) * g + h) * D + dd]);
+      den += w;
+    }
+    mp.o_dec[((size_t)r * mp.Hq + kvh * g + h) * D + dd] = __float2bfloat16_rn(num / den);
+  }
+}
+
+}  // namespace pod
+
+// =========================================================== host side (ABI)
+using namespace pod;
+
+namespace {
+
+thread_local int g_last_cuda = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda = (int)e;
+  return POD_ERR_CUDA;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int D>
+int configure_kernels() {
+  static bool done[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 64 && done[dev]) return POD_OK;
+  e = cudaFuncSetAttribute(pod_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemAlloc);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 64) done[dev] = true;
+  return POD_OK;
+}
+
+template <int D>
+int launch(const pod_attn_plan_t* pl, PodParams& prm, const MergeParams& mp, cudaStream_t st) {
+  int rc = configure_kernels<D>();
+  if (rc != POD_OK) return rc;
+  const size_t smem = Cfg<D>::kSmemAlloc;
+  if (pl->ev_start) cudaEventRecord(static_cast<cudaEvent_t>(pl->ev_start), st);
+  if (pl->cfg.flags & POD_FLAG_SEQUENTIAL) {
+    if (pl->n_pre > 0) {
+      prm.mode = kPrefillOnly;
+      prm.use_tmem = 1;
+      const int grid = pl->n_pre < pl->grid ? pl->n_pre : pl->grid;
+      pod_attn_kernel<D><<<grid, 128, smem, st>>>(prm);
+    }
+    if (pl->n_dec > 0) {
+      prm.mode = kDecodeOnly;
+      prm.use_tmem = 0;
+      pod_attn_kernel<D><<<pl->grid, 128, smem, st>>>(prm);
+    }
+  } else if (pl->n_pre > 0 || pl->n_dec > 0) {
+    prm.mode = kFused;
+    prm.use_tmem = pl->n_pre > 0 ? 1 : 0;
+    pod_attn_kernel<D><<<pl->grid, 128, smem, st>>>(prm);
+  }
+  if (pl->ev_stop) cudaEventRecord(static_cast<cudaEvent_t>(pl->ev_stop), st);
+  if (pl->n_merge > 0) pod_merge_kernel<D><<<pl->n_merge, 128, 0, st>>>(mp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return POD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pod_attn_status_string(int s) {
+  switch (s) {
+    case POD_OK: return "ok";
+    case POD_ERR_INVALID_ARG: return "invalid argument";
+    case POD_ERR_UNSUPPORTED: return "unsupported shape (head_dim 64/128, group <= 8, page 16)";
+    case POD_ERR_WORKSPACE: return "workspace too small";
+    case POD_ERR_CUDA: return "CUDA runtime error";
+    case POD_ERR_BOUNDS: return "block id out of range";
+    case POD_ERR_TIMEOUT: return "device wait timed out";
+    case POD_ERR_PLAN_MISMATCH: return "kv lengths disagree with the plan";
+    default: return "unknown status";
+  }
+}
+
+int pod_attn_last_cuda_error(void) { return g_last_cuda; }
+
+int pod_attn_plan(const pod_attn_config* cfg, int32_t prefill_qo_len, int32_t prefill_kv_len, int32_t num_decode,
+                  const int32_t* decode_kv_lens, pod_attn_plan_t** plan_out, size_t* workspace_bytes_out) {
+  if (!cfg || !plan_out) return POD_ERR_INVALID_ARG;
+  *plan_out = nullptr;
+  int sms = cfg->num_sms;
+  if (sms == 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  pod_attn_plan_t* pl = nullptr;
+  const int rc = pod_plan_build(cfg, sms, prefill_qo_len, prefill_kv_len, num_decode, decode_kv_lens, &pl);
+  if (rc != POD_OK) return rc;
+  pl->cfg.num_sms = sms;
+  *plan_out = pl;
+  if (workspace_bytes_out) *workspace_bytes_out = (size_t)pl->ws_bytes;
+  return POD_OK;
+}
+
+int pod_attn_plan_get_info(const pod_attn_plan_t* pl, pod_attn_plan_info* info) {
+  if (!pl || !info) return POD_ERR_INVALID_ARG;
+  info->num_prefill_items = pl->n_pre;
+  info->num_decode_items = pl->n_dec;
+  info->num_merge_items = pl->n_merge;
+  info->num_partials = pl->n_part;
+  info->ctas_per_sm = pl->ctas;
+  info->ratio_prefill = pl->ratio_p;
+  info->ratio_decode = pl->ratio_d;
+  info->chunk_pages = pl->chunk_pages;
+  info->num_sms = pl->num_sms;
+  info->grid = pl->grid;
+  info->workspace_bytes = pl->ws_bytes;
+  info->error_offset = 4LL * kErrorWord;
+  info->prefill_flops = pl->prefill_flops;
+  info->decode_flops = pl->decode_flops;
+  info->kv_bytes = pl->kv_bytes;
+  info->qo_bytes = pl->qo_bytes;
+  return POD_OK;
+}
+
+int pod_attn_plan_tables(const pod_attn_plan_t* pl, int32_t* pre, int32_t* dec, int32_t* merge) {
+  if (!pl) return POD_ERR_INVALID_ARG;
+  if (pre && !pl->pre.empty()) std::memcpy(pre, pl->pre.data(), pl->pre.size() * 4);
+  if (dec && !pl->dec.empty()) std::memcpy(dec, pl->dec.data(), pl->dec.size() * 4);
+  if (merge && !pl->merge.empty()) std::memcpy(merge, pl->merge.data(), pl->merge.size() * 4);
+  return POD_OK;
+}
+
+int pod_attn_upload(const pod_attn_plan_t* pl, void* ws, size_t ws_bytes, void* stream) {
+  if (!pl || !ws) return POD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return POD_ERR_INVALID_ARG;
+  if ((int64_t)ws_bytes < pl->ws_bytes) return POD_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kCountersBytes, st);
+  if (e == cudaSuccess && !pl->image.empty())
+    e = cudaMemcpyAsync(static_cast<uint8_t*>(ws) + kCountersBytes, pl->image.data(), pl->image.size(),
+                        cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return POD_OK;
+}
+
+int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q_decode, const void* k_cache,
+                 const void* v_cache, int64_t num_blocks, const int32_t* block_table, int32_t block_table_stride,
+                 const int32_t* kv_lens, float scale, void* o_prefill, void* o_decode, void* ws, size_t ws_bytes,
+                 int32_t* trace, void* stream) {
+  if (!pl || !ws) return POD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return POD_ERR_INVALID_ARG;
+  if ((int64_t)ws_bytes < pl->ws_bytes) return POD_ERR_WORKSPACE;
+  const int D = pl->cfg.head_dim, Hq = pl->cfg.num_q_heads, Hkv = pl->cfg.num_kv_heads;
+  const bool has_pre = pl->n_pre > 0, has_dec = pl->n_dec > 0;
+  if (has_pre && (!q_prefill || !o_prefill || !aligned16(q_prefill) || !aligned16(o_prefill)))
+    return POD_ERR_INVALID_ARG;
+  if (has_dec && (!q_decode || !o_decode || !aligned16(q_decode) || !aligned16(o_decode)))
+    return POD_ERR_INVALID_ARG;
+  if ((has_pre || has_dec) &&
+      (!k_cache || !v_cache || !aligned16(k_cache) || !aligned16(v_cache) || !block_table || num_blocks < 1))
+    return POD_ERR_INVALID_ARG;
+  if (block_table_stride < 1 || !(scale > 0.f) || scale != scale) return POD_ERR_INVALID_ARG;
+  if (num_blocks * Hkv * kPage >= (int64_t)INT32_MAX) return POD_ERR_UNSUPPORTED;
+  if ((pl->cfg.flags & POD_FLAG_TRACE) && !trace) return POD_ERR_INVALID_ARG;
+  if (!(has_pre || has_dec)) return POD_OK;
+
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return cuda_fail(cudaErrorNotSupported);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  PodParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)num_blocks * Hkv * kPage};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kPage};
+    const cuuint32_t es[2] = {1, 1};
+    CUresult r1 = enc(&prm.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_cache), dims, strides, box,
+                      es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r2 = enc(&prm.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(v_cache), dims, strides, box,
+                      es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r1 != CUDA_SUCCESS || r2 != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
+  }
+  if (has_pre) {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)pl->P};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kBM};
+    const cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = enc(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q_prefill), dims, strides, box,
+                     es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  prm.q_dec = static_cast<const __nv_bfloat16*>(q_decode);
+  prm.o_pre = static_cast<__nv_bfloat16*>(o_prefill);
+  prm.o_dec = static_cast<__nv_bfloat16*>(o_decode);
+  prm.block_table = block_table;
+  prm.kv_lens = kv_lens;
+  prm.counters = reinterpret_cast<int32_t*>(w);
+  prm.pre_items = reinterpret_cast<const int4*>(w + pl->off_pre);
+  prm.dec_items = reinterpret_cast<const int4*>(w + pl->off_dec);
+  prm.part_o = reinterpret_cast<float*>(w + pl->off_part_o);
+  prm.part_lse = reinterpret_cast<float*>(w + pl->off_part_lse);
+  prm.trace = (pl->cfg.flags & POD_FLAG_TRACE) ? trace : nullptr;
+  prm.bt_stride = block_table_stride;
+  prm.kv_rows = (int32_t)(num_blocks * Hkv * kPage);
+  prm.num_blocks = (int32_t)num_blocks;
+  prm.n_pre = pl->n_pre;
+  prm.n_dec = pl->n_dec;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.g = pl->g;
+  prm.P = pl->P;
+  prm.C = pl->C;
+  prm.B = pl->B;
+  prm.ratio_p = pl->ratio_p;
+  prm.ratio_d = pl->ratio_d;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+
+  MergeParams mp;
+  mp.items = reinterpret_cast<const int4*>(w + pl->off_merge);
+  mp.part_o = prm.part_o;
+  mp.part_lse = prm.part_lse;
+  mp.o_dec = prm.o_dec;
+  mp.n_merge = pl->n_merge;
+  mp.Hq = Hq;
+  mp.g = pl->g;
+
+  // counters (tickets, queue heads, error word) start at zero every run
+  cudaError_t e = cudaMemsetAsync(ws, 0, kCountersBytes, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return D == 128 ? launch<128>(pl, prm, mp, st) : launch<64>(pl, prm, mp, st);
+}
+
+int pod_attn_plan_set_events(pod_attn_plan_t* pl, void* ev_start, void* ev_stop) {
+  if (!pl) return POD_ERR_INVALID_ARG;
+  pl->ev_start = ev_start;
+  pl->ev_stop = ev_stop;
+  return POD_OK;
+}
+
+int pod_attn_event_create(void** ev_out) {
+  if (!ev_out) return POD_ERR_INVALID_ARG;
+  cudaEvent_t ev;
+  cudaError_t e = cudaEventCreate(&ev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *ev_out = ev;
+  return POD_OK;
+}
+
+int pod_attn_event_destroy(void* ev) {
+  if (!ev) return POD_OK;
+  cudaError_t e = cudaEventDestroy(static_cast<cudaEvent_t>(ev));
+  return e == cudaSuccess ? POD_OK : cuda_fail(e);
+}
+
+int pod_attn_event_elapsed_ms(void* a, void* b, float* ms) {
+  if (!a || !b || !ms) return POD_ERR_INVALID_ARG;
+  cudaError_t e = cudaEventElapsedTime(ms, static_cast<cudaEvent_t>(a), static_cast<cudaEvent_t>(b));
+  return e == cudaSuccess ? POD_OK : cuda_fail(e);
+}
+
+void pod_attn_plan_destroy(pod_attn_plan_t* pl) { delete pl; }
+
+}  // extern "C"

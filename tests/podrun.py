@@ -1,0 +1,46 @@
+"""Test/bench helper: move a synthetic batch to the GPU and run it through the
+C ABI.  Marshalling only (torch allocates device memory); no attention math."""
+from __future__ import annotations
+
+import numpy as np
+
+
+def bits_to_bf16(torch, a: np.ndarray, device="cuda"):
+    t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16))
+    return t.view(torch.bfloat16).to(device)
+
+
+class DeviceBatch:
+    def __init__(self, torch, b, device="cuda"):
+        self.b = b
+        w = b.workload
+        self.torch = torch
+        self.q_pre = bits_to_bf16(torch, b.q_prefill, device) if w.prefill_len else None
+        self.q_dec = bits_to_bf16(torch, b.q_decode, device) if w.num_decode else None
+        self.k = bits_to_bf16(torch, b.k_pool, device)
+        self.v = bits_to_bf16(torch, b.v_pool, device)
+        self.bt = torch.from_numpy(b.block_table).to(device)
+        self.lens = torch.from_numpy(b.kv_lens).to(device)
+        self.o_pre = torch.empty_like(self.q_pre) if self.q_pre is not None else None
+        self.o_dec = torch.empty_like(self.q_dec) if self.q_dec is not None else None
+
+    def plan(self, pod, **kw):
+        w = self.b.workload
+        P, C = w.prefill_len, w.prefill_ctx
+        return pod.Plan(w.num_q_heads, w.num_kv_heads, w.head_dim, P, C + P, self.b.decode_lens, **kw)
+
+    def workspace(self, plan):
+        return self.torch.zeros(max(plan.workspace_bytes, 256), dtype=self.torch.uint8, device=self.k.device)
+
+    def run(self, pod, plan, ws, trace=None, stream=None):
+        plan.run(self.q_pre, self.q_dec, self.k, self.v, self.b.num_blocks, self.bt, self.bt.shape[1], self.lens,
+                 self.b.scale, self.o_pre, self.o_dec, ws, trace=trace, stream=stream)
+
+    def outputs(self):
+        op = self.o_pre.float().cpu().numpy().astype(np.float64) if self.o_pre is not None else None
+        od = self.o_dec.float().cpu().numpy().astype(np.float64) if self.o_dec is not None else None
+        return op, od
+
+    def error_word(self, plan, ws):
+        off = plan.info.error_offset
+        return int(ws[off:off + 4].view(self.torch.int32).item())

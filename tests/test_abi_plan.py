@@ -1,0 +1,130 @@
+"""C-ABI library checks that need no GPU: it loads, exports every entry point
+that include/pod_attn.h declares, and its C++ planner reproduces the plan rule
+of oracle/plan_ref.py bit for bit (tables, split size, ratio), including the
+inputs it must reject."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from oracle.plan_ref import plan_ref, PlanError
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pod():
+    from prefill_decode_b200 import build
+    build.build()
+    import prefill_decode_b200 as m
+    m.lib()
+    return m
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "pod_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pod_attn_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol(pod):
+    names = _declared_functions()
+    assert len(names) >= 10
+    L = ctypes.CDLL(pod.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/pod_attn.h but not exported"
+    assert sorted(pod.EXPORTED) == names
+
+
+def test_status_strings(pod):
+    assert pod.status_string(0) == "ok"
+    assert "workspace" in pod.status_string(pod.POD_ERR_WORKSPACE)
+
+
+CONFIGS = [synth.tiny(), synth.llama3_8b_mix(), synth.long_context_mix(), synth.decode_heavy_mix()] + synth.sweep_points()
+
+
+def _lens(w):
+    return [int(x) for x in synth._draw_lengths(np.random.default_rng(w.seed), w)]
+
+
+def _compare(pod, Hq, Hkv, d, sms, P, KV, lens, **kw):
+    ref = plan_ref(Hq, Hkv, d, sms, P, KV, lens, **kw)
+    ratio = (kw.get("ratio_p", 0), kw.get("ratio_d", 0))
+    pl = pod.Plan(Hq, Hkv, d, P, KV, lens, num_sms=sms, ctas_per_sm=kw.get("ctas_per_sm", 0), ratio=ratio,
+                  max_waves=kw.get("max_waves", 0), min_chunk_pages=kw.get("min_chunk_pages", 0))
+    pre, dec, mer = pl.tables()
+    np.testing.assert_array_equal(pre, ref.prefill_items)
+    np.testing.assert_array_equal(dec, ref.decode_items)
+    np.testing.assert_array_equal(mer, ref.merge_items)
+    i = pl.info
+    assert (i.ctas_per_sm, i.ratio_prefill, i.ratio_decode, i.chunk_pages, i.num_partials) == (
+        ref.ctas_per_sm, ref.ratio_p, ref.ratio_d, ref.chunk_pages, ref.num_partials)
+    assert i.grid == sms * ref.ctas_per_sm
+    return pl
+
+
+@pytest.mark.parametrize("w", CONFIGS, ids=lambda w: w.name)
+def test_c_plan_matches_plan_ref(pod, w):
+    P, C = w.prefill_len, w.prefill_ctx
+    pl = _compare(pod, w.num_q_heads, w.num_kv_heads, w.head_dim, 148, P, C + P, _lens(w))
+    # algorithmic counts used by the roofline
+    L = sum(_lens(w))
+    assert pl.info.decode_flops == 4 * w.head_dim * w.num_q_heads * L
+    assert pl.info.kv_bytes == 4 * w.head_dim * w.num_kv_heads * ((C + P if P else 0) + L)
+    assert pl.info.prefill_flops == 4 * w.head_dim * w.num_q_heads * sum(C + i + 1 for i in range(P))
+
+
+def test_c_plan_matches_plan_ref_random(pod):
+    rng = np.random.default_rng(2024)
+    for _ in range(80):
+        Hkv = int(rng.choice([1, 2, 4, 8]))
+        g = int(rng.choice([1, 2, 4, 8]))
+        P = int(rng.choice([0, 1, 100, 128, 129, 513]))
+        C = int(rng.integers(0, 4000)) if P else 0
+        B = int(rng.integers(0 if P else 1, 50))
+        lens = [int(x) for x in rng.integers(1, 9000, size=B)]
+        kw = dict(ctas_per_sm=int(rng.choice([0, 1, 2])), max_waves=int(rng.choice([0, 1, 3])),
+                  min_chunk_pages=int(rng.choice([0, 1, 4, 16])),
+                  ratio_p=int(rng.choice([0, 0, 1, 2])), ratio_d=int(rng.choice([0, 0, 1, 3])))
+        _compare(pod, Hkv * g, Hkv, int(rng.choice([64, 128])), int(rng.integers(1, 200)), P, C + P, lens, **kw)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(Hq=30, Hkv=8), -1), (dict(Hq=32, Hkv=2), -2), (dict(d=96), -2), (dict(page=32), -2),
+    (dict(sms=600), -1), (dict(ctas=4), -1), (dict(P=10, KV=5), -1), (dict(lens=[0]), -1),
+    (dict(lens=[-3]), -1), (dict(lens=[1 << 25]), -1), (dict(ratio=(-1, 1)), -1),
+])
+def test_c_plan_rejects(pod, bad, code):
+    a = dict(Hq=32, Hkv=8, d=128, page=16, sms=148, ctas=0, P=64, KV=128, lens=[100, 200], ratio=(0, 0))
+    a.update(bad)
+    with pytest.raises(pod.PodError) as e:
+        pod.Plan(a["Hq"], a["Hkv"], a["d"], a["P"], a["KV"], a["lens"], num_sms=a["sms"], ctas_per_sm=a["ctas"],
+                 ratio=a["ratio"], page_size=a["page"])
+    assert e.value.status == code
+    with pytest.raises(PlanError):
+        plan_ref(a["Hq"], a["Hkv"], a["d"], a["sms"], a["P"], a["KV"], a["lens"], page_size=a["page"],
+                 ctas_per_sm=a["ctas"], ratio_p=a["ratio"][0], ratio_d=a["ratio"][1])
+
+
+def test_run_rejects_bad_host_arguments(pod):
+    """Argument validation happens on the host before any launch (no GPU needed)."""
+    pl = pod.Plan(4, 2, 64, 64, 192, [64, 100], num_sms=4)
+    ws = pl.workspace_bytes
+    L = pod.lib()
+    # null workspace
+    assert L.pod_attn_run(pl.handle, 16, 16, 16, 16, 10, 16, 4, None, 0.125, 16, 16, None, ws, None, None) == -1
+    # misaligned workspace
+    assert L.pod_attn_run(pl.handle, 16, 16, 16, 16, 10, 16, 4, None, 0.125, 16, 16, 0x1010, ws, None, None) == -1
+    # workspace too small
+    assert L.pod_attn_run(pl.handle, 16, 16, 16, 16, 10, 16, 4, None, 0.125, 16, 16, 0x1000, 256, None, None) == -3
+    # misaligned q pointer
+    assert L.pod_attn_run(pl.handle, 17, 16, 16, 16, 10, 16, 4, None, 0.125, 16, 16, 0x1000, ws, None, None) == -1
+    # bad scale
+    assert L.pod_attn_run(pl.handle, 16, 16, 16, 16, 10, 16, 4, None, -1.0, 16, 16, 0x1000, ws, None, None) == -1
+    # upload: too small / misaligned
+    assert L.pod_attn_upload(pl.handle, 0x1000, 256, None) == -3
+    assert L.pod_attn_upload(pl.handle, 0x1010, ws, None) == -1
