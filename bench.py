@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Bench: fused hybrid-batch (prefill + decode) attention on B200.
+
+Metric: hybrid-batch attention time in microseconds per batch (lower is
+better) and its fraction of the fused roofline
+max(prefill FLOPs / tensor peak, (KV + Q + O bytes) / HBM peak).
+
+One step = one ``pod_attn_run`` of the whole hybrid batch (counter reset, the
+persistent fused kernel, the LSE merge) on the Llama-3-8B-shaped workload
+(32 q / 8 kv heads, d = 128, prefill chunk 512 over 4096 prior tokens, 64
+decode requests with lengths uniform in [1024, 4096], 16-token pages), inputs
+resident in HBM.  The KV streamed per step (~0.67 GB) is larger than the 126 MB
+L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica of the batch (the path has no exchange step); the reported time is the
+max over ranks.  ``--impl reference`` times the CPU float64 oracle instead (on
+rank 0 only), on a bounded sample of the same batch, extrapolated per batch.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "hybrid-batch attention µs and % of fused max(tensor,HBM) roofline on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["prefill_decode_b200/csrc/pod_attn.cu", "prefill_decode_b200/csrc/pod_ptx.cuh",
+                  "prefill_decode_b200/csrc/pod_plan.h"]
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch of the fused kernel from a committed ncu summary,
+    valid only while the kernel sources are unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < 5:
+            time.sleep(0.02)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        inside = [p for (t, p) in self.samples if t0 <= t <= t1]
+        window = "timed region"
+        if not inside:
+            inside = [p for (t, p) in self.samples if t0 - 0.3 <= t <= t1 + 0.3]
+            window = "within 0.3 s of the timed region"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(p[1]) for p in inside if num(p[1]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in inside:
+            for n, v in zip(names, p[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(inside[0][2]),
+                "reasons": sorted(reasons), "samples": len(inside), "window": window,
+                "power_w_max": max((num(p[3]) or 0.0) for p in inside)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_oracle_time(b, decode_reqs, prefill_rows):
+    """Time the float64 oracle on a subset; return (seconds, decode part, prefill part, outputs)."""
+    from oracle import attention as A
+    w = b.workload
+    t0 = time.perf_counter()
+    od = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, w.num_kv_heads,
+                         requests=decode_reqs) if len(decode_reqs) else None
+    t1 = time.perf_counter()
+    op = A.attend_prefill(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_ctx, b.scale, w.num_kv_heads,
+                          rows=prefill_rows) if len(prefill_rows) else None
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1, od, op
+
+
+def extrapolate(b, decode_reqs, prefill_rows, t_dec, t_pre):
+    """Scale sampled oracle time to the whole batch by keys visited."""
+    L = b.decode_lens.astype(np.int64)
+    dec_scale = float(L.sum()) / max(1.0, float(L[list(decode_reqs)].sum())) if len(decode_reqs) else 0.0
+    C, P = b.prefill_ctx, b.prefill_len
+    keys_all = sum(C + i + 1 for i in range(P))
+    keys_s = sum(C + int(i) + 1 for i in prefill_rows)
+    pre_scale = keys_all / keys_s if keys_s else 0.0
+    return t_dec * dec_scale + t_pre * pre_scale
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        return 1
+
+
+def sample_sets(b, frac_den: int):
+    B, P = b.workload.num_decode, b.prefill_len
+    reqs = list(range(0, B, frac_den)) if B else []
+    rows = list(range(0, P, frac_den)) if P else []
+    return reqs, rows
+
+
+# ------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = synth.NAMED[args.workload]()
+    b = synth.make_batch(w)
+    reqs, rows = sample_sets(b, 8)
+    times = []
+    for i in range(args.warmup + args.steps):
+        td, tp, _, _ = cpu_oracle_time(b, reqs, rows)
+        if i >= args.warmup:
+            times.append(extrapolate(b, reqs, rows, td, tp) * 1e6)
+    v = float(np.mean(times))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w, b, "oracle"),
+            "cpu_baseline": {"value": v, "unit": "us", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"every 8th decode request ({len(reqs)}) and every 8th prefill row "
+                                       f"({len(rows)}), all heads; time scaled to the whole batch by keys visited"},
+            "e2e": {"value": v, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, b, mode):
+    L = b.decode_lens
+    return {"workload": w.name, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "prefill_len": w.prefill_len, "prefill_ctx": w.prefill_ctx,
+            "num_decode": w.num_decode, "decode_lens": f"{w.lens_kind}{list(w.lens_args)}, seed {w.seed}",
+            "sum_decode_len": int(L.sum()) if len(L) else 0, "page_size": 16, "mode": mode,
+            "l2": "no flush: inputs larger than L2 (the KV streamed per step exceeds 126 MB)"}
+
+
+# --------------------------------------------------------------------- ours
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama3_8b_mix", choices=sorted(synth.NAMED))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from prefill_decode_b200 import build
+    build.build()
+    import prefill_decode_b200 as pod
+    from tests.podrun import DeviceBatch
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = synth.NAMED[args.workload]()
+    b = synth.make_batch(w)
+    db = DeviceBatch(torch, b, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fused = db.plan(pod)
+    seq = db.plan(pod, flags=pod.POD_FLAG_SEQUENTIAL)
+    ws = db.workspace(fused)
+    ws_seq = db.workspace(seq)
+    fused.upload(ws, stream)
+    seq.upload(ws_seq, stream)
+    info = fused.info
+    launches_per_step = 1 + (1 if info.num_merge_items > 0 else 0)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def timed_loop(plan, wsp, K, per_step_events):
+        evs = [(pod.Event(), pod.Event()) for _ in range(K)] if per_step_events else []
+        for _ in range(args.warmup):
+            db.run(pod, plan, wsp, stream=stream)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        t_wall0 = time.time()
+        e0.record(stream)
+        for i in range(K):
+            if per_step_events:
+                plan.set_events(evs[i][0].handle, evs[i][1].handle)
+            db.run(pod, plan, wsp, stream=stream)
+        e1.record(stream)
+        barrier()
+        t_wall1 = time.time()
+        plan.set_events(None, None)
+        total_ms = e0.elapsed_time(e1)
+        kern = [a.elapsed_ms(c) for a, c in evs] if per_step_events else []
+        return total_ms, kern, (t_wall0, t_wall1)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    gpu_id = str(local)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    total_ms, kern_ms, (tw0, tw1) = timed_loop(fused, ws, args.steps, True)
+    clocks = sampler.summary(tw0, tw1)
+    seq_ms, seq_kern, _ = timed_loop(seq, ws_seq, max(50, args.steps // 4), True)
+    sampler.stop()
+    err_word = db.error_word(fused, ws)
+
+    us = max_over_ranks(total_ms * 1e3 / args.steps)
+    kern_us = max_over_ranks(float(np.mean(kern_ms)) * 1e3)
+    seq_us = max_over_ranks(seq_ms * 1e3 / max(50, args.steps // 4))
+    seq_kern_us = max_over_ranks(float(np.mean(seq_kern)) * 1e3)
+
+    # ------------------------------------------------------------- e2e
+    e2e = None
+    if not args.no_e2e:
+        host = {}
+        for name in ("q_pre", "q_dec", "k", "v", "bt", "lens"):
+            t = getattr(db, name)
+            if t is not None:
+                host[name] = t.cpu().pin_memory()
+        outs_host = {n: torch.empty(getattr(db, n).shape, dtype=getattr(db, n).dtype, pin_memory=True)
+                     for n in ("o_pre", "o_dec") if getattr(db, n) is not None}
+        h2d = sum(t.numel() * t.element_size() for t in host.values()) + info.table_bytes
+        d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+
+        def e2e_step():
+            for n, t in host.items():
+                getattr(db, n).copy_(t, non_blocking=True)
+            fused.upload(ws, stream)
+            db.run(pod, fused, ws, stream=stream)
+            for n, t in outs_host.items():
+                t.copy_(getattr(db, n), non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        barrier()
+        e2e_us = max_over_ranks(a0.elapsed_time(a1) * 1e3 / args.e2e_steps)
+        e2e = {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
+               "note": "pinned host Q, K/V pools, block table and lengths copied in, plan tables uploaded, "
+                       "outputs copied out, every step"}
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
+    # ------------------------------------------------------------ roofline
+    peaks, peak_src = load_peaks()
+    alg_bytes = info.kv_bytes + info.qo_bytes
+    t_hbm_us = alg_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6
+    t_tc_us = info.prefill_flops / (peaks["bf16_tflops"] * 1e12) * 1e6
+    bound = "hbm" if t_hbm_us >= t_tc_us else "tensor"
+    if bound == "hbm":
+        achieved = alg_bytes / (kern_us * 1e-6) / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved = info.prefill_flops / (kern_us * 1e-6) / 1e12
+        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+    traffic = load_traffic(w.name)
+
+    # ---------------------------------------------------------- CPU oracle
+    cpu = None
+    parity = None
+    if not args.no_cpu_baseline:
+        reqs, rows = sample_sets(b, 8)
+        td, tp, od, op = cpu_oracle_time(b, reqs, rows)
+        v = extrapolate(b, reqs, rows, td, tp) * 1e6
+        cpu = {"value": v, "unit": "us", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"every 8th decode request ({len(reqs)}) and every 8th prefill row ({len(rows)}), all "
+                         f"heads; measured {td + tp:.2f} s, scaled to the whole batch by keys visited",
+               "host_cpus": os.cpu_count()}
+        # the oracle outputs of that sample double as a parity spot check of the timed path
+        gp, gd = db.outputs()
+        e_dec = np.abs(gd[reqs] - od) if od is not None else np.zeros(1)
+        e_pre = np.abs(gp[rows] - op) if op is not None else np.zeros(1)
+        parity = {"max_abs": float(max(e_dec.max(), e_pre.max())),
+                  "mean_abs": float(np.concatenate([e_dec.ravel(), e_pre.ravel()]).mean()),
+                  "tolerance": {"max_abs": 2e-2, "mean_abs": 2e-3}}
+
+    line = {
+        "metric": METRIC, "value": us, "unit": "us", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(w, b, "fused"),
+        "fused_roofline": {"t_tensor_us": t_tc_us, "t_hbm_us": t_hbm_us, "t_roofline_us": max(t_tc_us, t_hbm_us),
+                           "frac_step": max(t_tc_us, t_hbm_us) / us, "frac_kernel": max(t_tc_us, t_hbm_us) / kern_us,
+                           "peaks": f"{peak_src}: HBM {peaks['hbm_gbs']} GB/s, bf16 {peaks['bf16_tflops']} TFLOP/s"},
+        "roofline": {"kernel": "pod_attn_kernel<128> (fused persistent)", "bound": bound, "achieved": achieved,
+                     "peak": peak, "unit": unit, "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": traffic, "algorithmic_bytes": int(alg_bytes),
+                     "algorithmic_flops_prefill": int(info.prefill_flops), "kernel_us": kern_us},
+        "sequential_us": seq_us, "sequential_kernels_us": seq_kern_us, "speedup_vs_sequential": seq_us / us,
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
+        "plan": {"prefill_items": info.num_prefill_items, "decode_items": info.num_decode_items,
+                 "merge_items": info.num_merge_items, "chunk_pages": info.chunk_pages,
+                 "ctas_per_sm": info.ctas_per_sm, "ratio": [info.ratio_prefill, info.ratio_decode],
+                 "grid": info.grid},
+        "device_error_word": err_word, "parity_sample": parity,
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

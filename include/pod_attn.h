@@ -102,6 +102,7 @@ typedef struct pod_attn_plan_info {
   int64_t decode_flops;       /* 4 d Hq sum_r L_r */
   int64_t kv_bytes;           /* 4 d Hkv (C + P + sum_r L_r): K and V read once */
   int64_t qo_bytes;           /* 4 d Hq (P + B): Q read and O written once */
+  int64_t table_bytes;        /* bytes pod_attn_upload copies host -> device */
 } pod_attn_plan_info;
 
 /* Build the schedule for one hybrid batch on the host (no device work).

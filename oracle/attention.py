@@ -34,14 +34,14 @@ PAGE = 16
 def gather_tokens(pool: np.ndarray, bt_row: np.ndarray, length: int, kv_head: int) -> np.ndarray:
     """Rows 0..length-1 of one request's K (or V) for one kv head, as float64 [length, d].
 
-    ``pool`` is float64 [num_blocks, Hkv, 16, d]; token j lives in block
-    bt_row[j // 16], slot j % 16."""
+    ``pool`` is [num_blocks, Hkv, 16, d], either bf16 bit patterns (uint16) or
+    floats; token j lives in block bt_row[j // 16], slot j % 16.  Only the
+    gathered tokens are upcast."""
     d = pool.shape[-1]
-    out = np.empty((length, d), dtype=np.float64)
-    for j in range(0, length, PAGE):
-        n = min(PAGE, length - j)
-        out[j:j + n] = pool[int(bt_row[j // PAGE]), kv_head, :n, :]
-    return out
+    npages = (length + PAGE - 1) // PAGE
+    blocks = np.asarray(bt_row[:npages], dtype=np.int64)
+    pages = pool[blocks, kv_head]                       # [npages, 16, d]
+    return _as_f64(pages.reshape(npages * PAGE, d)[:length])
 
 
 def attend_rows(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float, limits: Sequence[int]) -> np.ndarray:
@@ -71,7 +71,7 @@ def attend_decode(q_dec, k_pool, v_pool, block_table, kv_lens, scale: float, num
 
     Returns float64 [B, Hq, d] (or [len(requests), Hq, d] for a subset)."""
     q = _as_f64(q_dec)
-    kp, vp = _as_f64(k_pool), _as_f64(v_pool)
+    kp, vp = k_pool, v_pool
     B, Hq, d = q.shape
     g = Hq // num_kv_heads
     reqs = range(B) if requests is None else list(requests)
@@ -93,7 +93,7 @@ def attend_prefill(q_pre, k_pool, v_pool, block_table, prior_ctx: int, scale: fl
     q_pre [P, Hq, d]; chunk row i sees keys 0..C+i.  Returns float64 [P, Hq, d]
     (or [len(rows), Hq, d] for a subset of chunk rows)."""
     q = _as_f64(q_pre)
-    kp, vp = _as_f64(k_pool), _as_f64(v_pool)
+    kp, vp = k_pool, v_pool
     P, Hq, d = q.shape
     C = int(prior_ctx)
     g = Hq // num_kv_heads

@@ -45,7 +45,7 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_prefill_items", "num_decode_items", "num_merge_items", "num_partials", "ctas_per_sm",
         "ratio_prefill", "ratio_decode", "chunk_pages", "num_sms", "grid")] + [(n, ctypes.c_int64) for n in (
-            "workspace_bytes", "error_offset", "prefill_flops", "decode_flops", "kv_bytes", "qo_bytes")]
+            "workspace_bytes", "error_offset", "prefill_flops", "decode_flops", "kv_bytes", "qo_bytes", "table_bytes")]
 
 
 class PodError(RuntimeError):

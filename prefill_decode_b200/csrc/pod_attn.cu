@@ -742,6 +742,7 @@ int pod_attn_plan_get_info(const pod_attn_plan_t* pl, pod_attn_plan_info* info) 
   info->decode_flops = pl->decode_flops;
   info->kv_bytes = pl->kv_bytes;
   info->qo_bytes = pl->qo_bytes;
+  info->table_bytes = (int64_t)pl->image.size();
   return POD_OK;
 }
 
