@@ -164,6 +164,36 @@ int pod_attn_event_create(void** ev_out);
 int pod_attn_event_destroy(void* ev);
 int pod_attn_event_elapsed_ms(void* ev_start, void* ev_stop, float* ms_out);
 
+/* Size of the fixed device workspace used by pod_attn_run_static (8 MiB). */
+#define POD_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* pod_attn_run without a caller-provided workspace.  The paper has no
+ * counterpart: this exists for callers that cannot allocate device memory,
+ * such as a plugin inside an inference engine that keeps (almost) all HBM in
+ * its own pools and offers no workspace hook, or a latency-critical caller
+ * that cannot pay for cudaMalloc's implicit device synchronisation.
+ * Instead of `workspace`, it uses a file-scope device array of
+ * POD_STATIC_SCRATCH_BYTES that every GPU which loads the library holds until
+ * the process exits; it allocates nothing.  Arguments, layouts and the async
+ * behaviour are those of pod_attn_run (no trace).
+ *  - The first call on a device looks up the array's device address for that
+ *    device (cudaGetSymbolAddress); make that first call before any stream
+ *    capture.
+ *  - Every call re-copies the plan's tables into the array and zeroes its
+ *    counters; the array keeps the last call's contents otherwise.
+ *  - All calls on a device share the one array: calls that overlap on the GPU
+ *    (other streams, other host threads) race and corrupt each other.
+ *    Serialise them, e.g. on one stream.
+ * Errors: POD_ERR_WORKSPACE if the plan needs more than
+ * POD_STATIC_SCRATCH_BYTES (see pod_attn_plan_info.workspace_bytes); otherwise
+ * those of pod_attn_upload and pod_attn_run. */
+int pod_attn_run_static(const pod_attn_plan_t* plan,
+                        const void* q_prefill, const void* q_decode,
+                        const void* k_cache, const void* v_cache, int64_t num_blocks,
+                        const int32_t* block_table, int32_t block_table_stride,
+                        const int32_t* kv_lens, float scale,
+                        void* o_prefill, void* o_decode, void* stream);
+
 /* Release a plan (null is allowed). */
 void pod_attn_plan_destroy(pod_attn_plan_t* plan);
 

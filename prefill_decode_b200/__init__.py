@@ -31,7 +31,7 @@ POD_FLAG_TRACE = 2
 EXPORTED = [
     "pod_attn_plan", "pod_attn_plan_get_info", "pod_attn_plan_tables", "pod_attn_upload", "pod_attn_run",
     "pod_attn_plan_set_events", "pod_attn_event_create", "pod_attn_event_destroy", "pod_attn_event_elapsed_ms",
-    "pod_attn_plan_destroy", "pod_attn_status_string", "pod_attn_last_cuda_error",
+    "pod_attn_plan_destroy", "pod_attn_status_string", "pod_attn_last_cuda_error", "pod_attn_run_static",
 ]
 
 
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
         L.pod_attn_status_string.argtypes = [ctypes.c_int]
         L.pod_attn_status_string.restype = ctypes.c_char_p
         L.pod_attn_last_cuda_error.argtypes = []
+        L.pod_attn_run_static.argtypes = [vp, vp, vp, vp, vp, i64, vp, i32, vp, ctypes.c_float, vp, vp, vp]
         for n in EXPORTED:
             if n not in ("pod_attn_plan_destroy", "pod_attn_status_string"):
                 getattr(L, n).restype = ctypes.c_int

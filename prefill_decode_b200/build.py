@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpod_attn.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("pod_attn.cu", "plan.cpp")]
+SOURCES = [os.path.join(CSRC, f) for f in ("pod_attn.cu", "plan.cpp", "pod_static.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in ("pod_plan.h", "pod_ptx.cuh")] + [os.path.join(INCLUDE, "pod_attn.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
