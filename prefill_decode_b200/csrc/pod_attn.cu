@@ -34,8 +34,7 @@
 namespace pod {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a healthy wait takes microseconds
-constexpr uint32_t kTmemCols = 256;                // S (64 cols) at 0, O tile (d cols) at 128
-constexpr uint32_t kTmemS = 0;
+constexpr uint32_t kTmemCols = 256;                // S double buffer (2 x 64 cols) at 0, O (d cols) at 128
 constexpr uint32_t kTmemO = 128;
 
 enum Mode : int32_t { kFused = 0, kPrefillOnly = 1, kDecodeOnly = 2 };
@@ -67,21 +66,46 @@ struct alignas(64) PodParams {
   float scale_log2;        // softmax scale * log2(e)
 };
 
+constexpr int kThreads = 192;        // warps 0-3: softmax (prefill) / decode units; warp 4: MMA; warp 5: TMA
+constexpr int kMmaWarp = 4;
+constexpr int kTmaWarp = 5;
+
+// mbarrier slots in the CTA control block
+enum : int {
+  kBarQ = 0,        // Q tile landed (TMA)                                    count 1 + tx
+  kBarKFull = 1,    // [3] K tile landed (TMA)                                count 1 + tx
+  kBarKEmpty = 4,   // [3] K slot free again: its P.V finished (MMA commit)   count 1
+  kBarVFull = 7,    // [2] V tile landed (TMA)                                count 1 + tx
+  kBarVEmpty = 9,   // [2] V slot free again (MMA commit)                     count 1
+  kBarSFull = 11,   // [2] S tile ready in TMEM (MMA commit)                  count 1
+  kBarSFree = 13,   // [2] S tile read out by the 4 softmax warps             count 4
+  kBarPFull = 15,   // [2] P tile written (and O rescaled) by 128 rows        count 128
+  kBarODone = 17,   // P.V MMA of a tile finished (MMA commit)                count 1
+  kBarDecode = 18,  // [kWarpsPerCta * kNS] decode page rings                 count 1 + tx
+};
+
 template <int D>
 struct Cfg {
   static constexpr int kHalves = D / 64;                      // 128-byte swizzle atoms along d
   static constexpr int kQBytes = kBM * D * 2;                 // 128 query rows
-  static constexpr int kKTile = kBN * D * 2;                  // 64 keys
-  static constexpr int kStage = 2 * kKTile;                   // K + V
-  static constexpr bool kPAliasK = (kBN * kBM * 2 <= kKTile); // P [128 x 64] fits in the spent K tile
-  static constexpr int kPrefillSmem = kQBytes + 2 * kStage + (kPAliasK ? 0 : kBM * kBN * 2);
+  static constexpr int kKTile = kBN * D * 2;                  // 64 keys of K (or V)
+  static constexpr int kKSlots = 3;                           // K ring: two tiles of lead
+  static constexpr int kVSlots = 2;                           // V ring: two tiles of lead
+  static constexpr int kPBytes = kBM * kBN * 2;               // P tile [128 x 64] bf16
+  static constexpr bool kPAliasK = (kPBytes <= kKTile);       // P is written over its spent K tile
+  static constexpr int kOffK = kQBytes;
+  static constexpr int kOffV = kOffK + kKSlots * kKTile;
+  static constexpr int kOffP = kOffV + kVSlots * kKTile;
+  static constexpr int kPrefillSmem = kOffP + (kPAliasK ? 0 : 2 * kPBytes);
   static constexpr int kPageBytes = kPage * D * 2;            // one 16-token page of one kv head
   static constexpr int kDecStage = 2 * kPageBytes;            // K page + V page
   static constexpr int kNS = (kPrefillSmem / kWarpsPerCta) / kDecStage;   // decode ring depth per warp
   static constexpr int kSmem = kPrefillSmem;
-  // + 1024 slack for 1024-byte alignment; at least 80 KB so that no more than two
-  // CTAs (2 x 256 TMEM columns) can ever share an SM
-  static constexpr int kSmemAlloc = (kSmem + 1024) > 80 * 1024 ? (kSmem + 1024) : 80 * 1024;
+  static constexpr int kNumBars = kBarDecode + kWarpsPerCta * kNS;
+  static constexpr int kCtrlBytes = 512;                      // barriers, TMEM address, broadcast slots
+  static_assert(kNumBars * 8 + 32 <= kCtrlBytes, "control block too small");
+  // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) can share an SM
+  static constexpr int kSmemAlloc = (kSmem + kCtrlBytes) > 80 * 1024 ? (kSmem + kCtrlBytes) : 80 * 1024;
 };
 static_assert(Cfg<128>::kNS >= 3 && Cfg<64>::kNS >= 3, "decode ring too shallow");
 
@@ -99,122 +123,247 @@ __device__ __forceinline__ int kv_row(const PodParams& p, int blk, int kvh) {
   return (blk * p.Hkv + kvh) * kPage;
 }
 
-struct PrefillState {
-  uint32_t q_phase;
-  uint32_t kv_phase[2];
-  uint32_t mma_phase;
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int D>
+struct PrefillSmem {
+  uint8_t* base;
+  __device__ uint8_t* q() const { return base; }
+  __device__ uint8_t* k(uint32_t t) const { return base + Cfg<D>::kOffK + (t % Cfg<D>::kKSlots) * Cfg<D>::kKTile; }
+  __device__ uint8_t* v(uint32_t t) const { return base + Cfg<D>::kOffV + (t % Cfg<D>::kVSlots) * Cfg<D>::kKTile; }
+  __device__ uint8_t* pt(uint32_t t) const {
+    return Cfg<D>::kPAliasK ? k(t) : base + Cfg<D>::kOffP + (t & 1u) * Cfg<D>::kPBytes;
+  }
 };
 
-// Load the 64-key tile `kb` (4 pages x d/64 halves of K and V) into stage `s`.
+// TMA warp: tensor-map rows of the 4 pages of key tile kb (lanes 0..3 look the
+// block ids up in parallel; pages past kv_end read past the tensor's end =
+// zeros).  Returns the row of page `lane & 3` in every lane.
+__device__ __forceinline__ int tile_page_row(const PodParams& p, int kb, int kvh, int kv_end, int lane) {
+  const int gp = kb * (kBN / kPage) + (lane & 3);
+  int row = p.kv_rows;
+  if (lane < 4 && gp * kPage < kv_end) row = kv_row(p, __ldg(&p.block_table[gp]), kvh);
+  return row;
+}
+
 template <int D>
-__device__ __forceinline__ void prefill_issue_tile(const PodParams& p, uint8_t* stage, uint64_t* bar, int kb,
-                                                   int kvh, int kv_end) {
+__device__ __forceinline__ void issue_tile(const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int row_lane,
+                                           int lane) {
   using CF = Cfg<D>;
-  mbar_arrive_expect_tx(bar, CF::kStage);
+  int rows[kBN / kPage];
 #pragma unroll
-  for (int pi = 0; pi < kBN / kPage; ++pi) {
-    const int gp = kb * (kBN / kPage) + pi;
-    int row = p.kv_rows;                       // pages past the request's end read as zeros
-    if (gp * kPage < kv_end) row = kv_row(p, __ldg(&p.block_table[gp]), kvh);
+  for (int pi = 0; pi < kBN / kPage; ++pi) rows[pi] = __shfl_sync(0xffffffffu, row_lane, pi);
+  if (lane == 0) {
+    mbar_arrive_expect_tx(bar, CF::kKTile);
 #pragma unroll
-    for (int h = 0; h < CF::kHalves; ++h) {
-      tma_load_2d(stage + h * (kBN * 128) + pi * (kPage * 128), &p.tm_k, bar, h * 64, row);
-      tma_load_2d(stage + CF::kKTile + h * (kBN * 128) + pi * (kPage * 128), &p.tm_v, bar, h * 64, row);
-    }
+    for (int pi = 0; pi < kBN / kPage; ++pi)
+#pragma unroll
+      for (int h = 0; h < CF::kHalves; ++h)
+        tma_load_2d(dst + h * (kBN * 128) + pi * (kPage * 128), map, bar, h * 64, rows[pi]);
   }
 }
 
-// One prefill work item: rows q0..q0+127 of query head qh against keys
-// 0..kv_end-1 of request 0 with the bottom-right causal mask.  All 128 threads;
-// thread t owns tile row t (TMEM lane t).  Returns false if a wait expired.
+// TMA warp of one prefill item: Q, then K into a 3-deep ring and V into a
+// 2-deep ring, refilling a slot as soon as the MMA warp reports its P.V done.
+// `t0` = key tiles this CTA processed before this item (it indexes every ring
+// and mbarrier phase).
 template <int D>
-__device__ bool prefill_item(const PodParams& p, int item, uint8_t* smem, uint64_t* bars, uint32_t tmem,
-                             PrefillState& st) {
+__device__ bool prefill_tma(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t t0) {
   using CF = Cfg<D>;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int4 it = __ldg(&p.pre_items[item]);
+  const int lane = threadIdx.x & 31;
   const int q0 = it.x, qh = it.y, kv_end = it.z;
   const int kvh = qh / p.g;
   const int nkb = (kv_end + kBN - 1) / kBN;
-  uint64_t* bar_q = &bars[0];
-  uint64_t* bar_kv = &bars[1];
-  uint64_t* bar_mma = &bars[3];
-  uint8_t* sQ = smem;
-  uint8_t* stage0 = smem + CF::kQBytes;
-
-  if (tid == 0) {
-    if (p.kv_lens && __ldg(&p.kv_lens[0]) < kv_end) record_error(p, POD_ERR_PLAN_MISMATCH, item);
-    mbar_arrive_expect_tx(bar_q, CF::kQBytes);
+  const PrefillSmem<D> sm{smem};
+  if (lane == 0) {
+    if (p.kv_lens && __ldg(&p.kv_lens[0]) < kv_end) record_error(p, POD_ERR_PLAN_MISMATCH, 0);
+    mbar_arrive_expect_tx(&bars[kBarQ], CF::kQBytes);
 #pragma unroll
-    for (int h = 0; h < CF::kHalves; ++h) tma_load_3d(sQ + h * (kBM * 128), &p.tm_q, bar_q, h * 64, qh, q0);
-    prefill_issue_tile<D>(p, stage0, &bar_kv[0], 0, kvh, kv_end);
+    for (int h = 0; h < CF::kHalves; ++h) tma_load_3d(sm.q() + h * (kBM * 128), &p.tm_q, &bars[kBarQ], h * 64, qh, q0);
   }
+  for (int j = 0; j < nkb && j < CF::kKSlots; ++j) {
+    const uint32_t t = t0 + j;
+    const int r = tile_page_row(p, j, kvh, kv_end, lane);
+    issue_tile<D>(&p.tm_k, sm.k(t), &bars[kBarKFull + t % 3], r, lane);
+    if (j < CF::kVSlots) issue_tile<D>(&p.tm_v, sm.v(t), &bars[kBarVFull + (t & 1u)], r, lane);
+  }
+  for (int j = 0; j + CF::kVSlots < nkb; ++j) {
+    const uint32_t t = t0 + j;
+    const bool more_k = j + CF::kKSlots < nkb;
+    const int rk = more_k ? tile_page_row(p, j + CF::kKSlots, kvh, kv_end, lane) : 0;
+    const int rv = tile_page_row(p, j + CF::kVSlots, kvh, kv_end, lane);
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarVEmpty + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs))) return false;
+    issue_tile<D>(&p.tm_v, sm.v(t + CF::kVSlots), &bars[kBarVFull + (t & 1u)], rv, lane);
+    if (more_k) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKEmpty + t % 3], (t / 3) & 1u, kWaitLimitNs))) return false;
+      issue_tile<D>(&p.tm_k, sm.k(t + CF::kKSlots), &bars[kBarKFull + t % 3], rk, lane);
+    }
+  }
+  return true;
+}
 
-  const uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false, false);
-  const uint32_t idesc_o = idesc_bf16_f32(kBM, D, false, true);
-  const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
-  const int row = tid;                                   // tile row
-  const int row_limit = min(p.C + q0 + row + 1, kv_end); // keys 0..row_limit-1 are visible
-  float o[D];
+// MMA warp of one prefill item (lane 0 issues): S_t = Q K_t^T into TMEM buffer
+// t&1 one tile ahead of the softmax; O += P_t V_t once P_t is written; each
+// P.V commit frees the tile's K and V slots and signals O.
+template <int D>
+__device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t tmem, uint32_t t0,
+                            uint32_t nq) {
+  using CF = Cfg<D>;
+  const int lane = threadIdx.x & 31;
+  const int kv_end = it.z;
+  const int nkb = (kv_end + kBN - 1) / kBN;
+  const PrefillSmem<D> sm{smem};
+  constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false, false);
+  constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, false, true);
+  // descriptors of the slot bases; a byte offset b within a slot adds b >> 4
+  const uint64_t dq = sdesc_sw128(smem_u32(sm.q()), 16, 1024);
+  const uint64_t dk0 = sdesc_sw128(smem_u32(smem + CF::kOffK), 16, 1024);
+  const uint64_t dv0 = sdesc_sw128(smem_u32(smem + CF::kOffV), kBN * 128, 1024);
+  const uint64_t dp0 = sdesc_sw128(smem_u32(CF::kPAliasK ? smem + CF::kOffK : smem + CF::kOffP), 16, 1024);
+
+  auto issue_s = [&](uint32_t t) {
+    const uint64_t dk = dk0 + (uint64_t)(((t % CF::kKSlots) * CF::kKTile) >> 4);
 #pragma unroll
-  for (int c = 0; c < D; ++c) o[c] = 0.f;
-  float m = -INFINITY, l = 0.f;
-  bool ok = true;
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t aoff = ((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4;
+      const uint32_t boff = ((kk >> 2) * (kBN * 128) + (kk & 3) * 32) >> 4;
+      umma_bf16(tmem + (t & 1u) * kBN, dq + aoff, dk + boff, idesc_s, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&bars[kBarSFull + (t & 1u)]);
+  };
 
-  for (int kb = 0; kb < nkb; ++kb) {
-    const int s = kb & 1;
-    uint8_t* sK = stage0 + s * CF::kStage;
-    uint8_t* sV = sK + CF::kKTile;
-    uint8_t* sP = CF::kPAliasK ? sK : (stage0 + 2 * CF::kStage);
-    if (tid == 0) {
-      bool w = true;
-      if (kb == 0) w = mbar_wait(bar_q, st.q_phase, kWaitLimitNs);
-      w = w && mbar_wait(&bar_kv[s], st.kv_phase[s], kWaitLimitNs);
-      if (w) {
+  bool w = mbar_wait(&bars[kBarQ], nq & 1u, kWaitLimitNs) &&
+           mbar_wait(&bars[kBarKFull + t0 % 3], (t0 / 3) & 1u, kWaitLimitNs);
+  if (t0 >= 2) w = w && mbar_wait(&bars[kBarSFree + (t0 & 1u)], ((t0 - 2) >> 1) & 1u, kWaitLimitNs);
+  if (!__all_sync(0xffffffffu, w)) return false;
+  if (lane == 0) {
+    tc_fence_after();
+    issue_s(t0);
+  }
+  __syncwarp();
+  for (int j = 0; j < nkb; ++j) {
+    const uint32_t t = t0 + j;
+    if (j + 1 < nkb) {           // S of the next tile runs while the softmax works on this one
+      const uint32_t tn = t + 1;
+      bool ws = mbar_wait(&bars[kBarKFull + tn % 3], (tn / 3) & 1u, kWaitLimitNs);
+      if (tn >= 2) ws = ws && mbar_wait(&bars[kBarSFree + (tn & 1u)], ((tn - 2) >> 1) & 1u, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ws)) return false;
+      if (lane == 0) {
         tc_fence_after();
-        const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK);
+        issue_s(tn);
+      }
+      __syncwarp();
+    }
+    bool wp = mbar_wait(&bars[kBarVFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs) &&
+              mbar_wait(&bars[kBarPFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs);
+    if (!__all_sync(0xffffffffu, wp)) return false;
+    const int valid = kv_end - j * kBN;
+    if (valid < kBN) {           // V rows past the request's end may hold anything: zero them
+      uint8_t* vt = sm.v(t);
+      for (int i = lane; i < (kBN - valid) * CF::kHalves * 8; i += 32) {
+        const int chunk = i & 7, rh = i >> 3;
+        const int key = valid + rh % (kBN - valid), h = rh / (kBN - valid);
+        *reinterpret_cast<uint4*>(vt + h * (kBN * 128) + key * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
+    if (lane == 0) {
+      tc_fence_after();
+      const uint64_t dp = dp0 + (uint64_t)((CF::kPAliasK ? (t % CF::kKSlots) * CF::kKTile : (t & 1u) * CF::kPBytes) >> 4);
+      const uint64_t dv = dv0 + (uint64_t)(((t & 1u) * CF::kKTile) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(ka + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024);
-          umma_bf16(tmem + kTmemS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_mma);
-        if (kb + 1 < nkb) prefill_issue_tile<D>(p, stage0 + (s ^ 1) * CF::kStage, &bar_kv[s ^ 1], kb + 1, kvh, kv_end);
-      } else {
-        record_error(p, POD_ERR_TIMEOUT, 1);
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        umma_bf16(tmem + kTmemO, dp + (uint64_t)((kk * 32) >> 4), dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_o,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(&bars[kBarODone]);
+      umma_commit(&bars[kBarKEmpty + t % 3]);
+      umma_commit(&bars[kBarVEmpty + (t & 1u)]);
+    }
+    __syncwarp();
+  }
+  return true;
+}
+
+// Softmax warps of one prefill item (threads 0..127, thread = tile row = TMEM
+// lane).  Per key tile: read S_t from TMEM, mask (bottom-right causal), online
+// softmax in the exp2 domain with a lazily updated row max (O in TMEM is
+// rescaled only when the max grows by more than 2^8), write P_t as bf16 in the
+// K-major 128B-swizzled layout; finally O / l -> bf16 -> global.
+template <int D>
+__device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t tmem,
+                                uint32_t t0) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q0 = it.x, qh = it.y, kv_end = it.z;
+  const int nkb = (kv_end + kBN - 1) / kBN;
+  const PrefillSmem<D> sm{smem};
+  const int row = tid;
+  const int row_limit = min(p.C + q0 + row + 1, kv_end);
+  const int full_tiles = (p.C + q0 + 1) / kBN;   // tiles visible to every row of this item
+  const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
+  const float sl2 = p.scale_log2;
+  float m = -INFINITY, l = 0.f;
+  for (int j = 0; j < nkb; ++j) {
+    const uint32_t t = t0 + j;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs))) return false;
+    tc_fence_after();
+    float s[kBN];
+    tmem_ld32(tmem + t_lane + (t & 1u) * kBN, s);
+    tmem_ld32(tmem + t_lane + (t & 1u) * kBN + 32, s + 32);
+    tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[kBarSFree + (t & 1u)]);
+    float mx = -INFINITY;
+    if (j < full_tiles) {
+#pragma unroll
+      for (int k = 0; k < kBN; ++k) {
+        s[k] *= sl2;
+        mx = fmaxf(mx, s[k]);
+      }
+    } else {
+      const int lim = row_limit - j * kBN;
+#pragma unroll
+      for (int k = 0; k < kBN; ++k) {
+        s[k] = k < lim ? s[k] * sl2 : -INFINITY;
+        mx = fmaxf(mx, s[k]);
       }
     }
-    if (kb == 0) st.q_phase ^= 1;
-    st.kv_phase[s] ^= 1;
-
-    // ---- S tile -> online softmax -> P (bf16, K-major 128B-swizzled in smem)
-    bool w1 = mbar_wait(bar_mma, st.mma_phase, kWaitLimitNs);
-    st.mma_phase ^= 1;
-    __syncwarp();
-    tc_fence_after();
-    float sv[kBN];
-    tmem_ld32(tmem + t_lane + kTmemS, sv);
-    tmem_ld32(tmem + t_lane + kTmemS + 32, sv + 32);
-    tmem_wait_ld();
-    const int lim = row_limit - kb * kBN;
-    float mx = -INFINITY;
+    if (j == 0) {
+      m = mx;
+    } else {
+      const bool need = mx > m + 8.f;
+      if (__any_sync(0xffffffffu, need)) {
+        // O holds the P.V sums of the earlier tiles: wait for the last one, then rescale
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone], (t - 1) & 1u, kWaitLimitNs))) return false;
+        tc_fence_after();
+        const float m_new = need ? mx : m;
+        const float alpha = ex2(m - m_new);
 #pragma unroll
-    for (int j = 0; j < kBN; ++j) {
-      sv[j] = (j < lim) ? sv[j] * p.scale_log2 : -INFINITY;
-      mx = fmaxf(mx, sv[j]);
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(tmem + t_lane + kTmemO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(tmem + t_lane + kTmemO + c * 32, o);
+        }
+        tmem_wait_st();
+        l *= alpha;
+        m = m_new;
+      }
     }
-    const float m_new = fmaxf(m, mx);
-    const float alpha = ex2(m - m_new);
     float rs = 0.f;
-    uint8_t* prow = sP + row * 128;
+    uint8_t* prow = sm.pt(t) + row * 128;
 #pragma unroll
     for (int c = 0; c < kBN / 8; ++c) {
       float e[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        e[j] = ex2(sv[c * 8 + j] - m_new);
-        rs += e[j];
+      for (int k = 0; k < 8; ++k) {
+        e[k] = ex2(s[c * 8 + k] - m);
+        rs += e[k];
       }
       uint4 v;
       v.x = pack_bf16(e[0], e[1]);
@@ -223,75 +372,35 @@ __device__ bool prefill_item(const PodParams& p, int item, uint8_t* smem, uint64
       v.w = pack_bf16(e[6], e[7]);
       *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v;
     }
-    l = l * alpha + rs;
-    m = m_new;
-    // zero V rows past kv_end in the last tile (they may hold anything)
-    const int valid_keys = kv_end - kb * kBN;
-    if (valid_keys < kBN) {
-      if (!mbar_wait(&bar_kv[s], st.kv_phase[s] ^ 1, kWaitLimitNs)) w1 = false;
-      const int nz = (kBN - valid_keys) * CF::kHalves * 8;   // 16-byte chunks to clear
-      for (int i = tid; i < nz; i += 128) {
-        const int chunk = i & 7, rh = i >> 3;
-        const int key = valid_keys + rh % (kBN - valid_keys), h = rh / (kBN - valid_keys);
-        *reinterpret_cast<uint4*>(sV + h * (kBN * 128) + key * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
-      }
-    }
+    l += rs;
     fence_proxy_async_smem();
     tc_fence_before();
-    if (__syncthreads_or(!w1)) {
-      ok = false;
-      break;
-    }
-    // ---- O tile = P V (fresh accumulator each key tile)
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t pa = smem_u32(sP), va = smem_u32(sV);
-#pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk) {
-        const uint64_t ad = sdesc_sw128(pa + kk * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(va + kk * (16 * 128), kBN * 128, 1024);
-        umma_bf16(tmem + kTmemO, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
-      }
-      umma_commit(bar_mma);
-    }
-    const bool w2 = mbar_wait(bar_mma, st.mma_phase, kWaitLimitNs);
-    st.mma_phase ^= 1;
-    __syncwarp();
-    tc_fence_after();
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      float ov[32];
-      tmem_ld32(tmem + t_lane + kTmemO + c * 32, ov);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) o[c * 32 + j] = o[c * 32 + j] * alpha + ov[j];
-    }
-    tc_fence_before();
-    if (__syncthreads_or(!w2)) {
-      ok = false;
-      break;
-    }
+    mbar_arrive(&bars[kBarPFull + (t & 1u)]);
   }
-  if (!ok) {
-    if (tid == 0) record_error(p, POD_ERR_TIMEOUT, 2);
-    return false;
-  }
-  // ---- epilogue: O / l -> bf16, one 2*D-byte row per thread
+  // epilogue: O / l -> bf16, one 2*D-byte row per thread
+  const uint32_t tl = t0 + nkb - 1;
+  if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone], tl & 1u, kWaitLimitNs))) return false;
+  tc_fence_after();
   const int q = q0 + row;
-  if (q < p.P) {
-    const float inv = 1.f / l;
-    uint4* dst = reinterpret_cast<uint4*>(p.o_pre + ((size_t)q * p.Hq + qh) * D);
+  const float inv = 1.f / l;
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      uint4 v;
-      v.x = pack_bf16(o[c * 8 + 0] * inv, o[c * 8 + 1] * inv);
-      v.y = pack_bf16(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv);
-      v.z = pack_bf16(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv);
-      v.w = pack_bf16(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
-      dst[c] = v;
+  for (int c = 0; c < D / 32; ++c) {
+    float o[32];
+    tmem_ld32(tmem + t_lane + kTmemO + c * 32, o);
+    tmem_wait_ld();
+    if (q < p.P) {
+      uint4* dst = reinterpret_cast<uint4*>(p.o_pre + ((size_t)q * p.Hq + qh) * D + c * 32);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint4 v;
+        v.x = pack_bf16(o[k * 8 + 0] * inv, o[k * 8 + 1] * inv);
+        v.y = pack_bf16(o[k * 8 + 2] * inv, o[k * 8 + 3] * inv);
+        v.z = pack_bf16(o[k * 8 + 4] * inv, o[k * 8 + 5] * inv);
+        v.w = pack_bf16(o[k * 8 + 6] * inv, o[k * 8 + 7] * inv);
+        dst[k] = v;
+      }
     }
   }
-  (void)lane;
   return true;
 }
 
@@ -504,21 +613,30 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
 }
 
 // --------------------------------------------------------- persistent kernel
+// Grid = SMs x CTAs/SM.  Each CTA takes one ticket from its SM's counter; the
+// ticket fixes its home role (prefill iff t mod (p+d) < p).  The CTA drains
+// its home queue, then the other one; no CTA ever waits for another.
 template <int D>
-__global__ void __launch_bounds__(128, 2) pod_attn_kernel(const __grid_constant__ PodParams p) {
+__global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_constant__ PodParams p) {
   using CF = Cfg<D>;
-  extern __shared__ uint8_t dyn_smem[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[4 + kWarpsPerCta * CF::kNS];
-  __shared__ uint32_t tmem_holder;
-  __shared__ int sh_home, sh_item;
-  __shared__ volatile int sh_abort;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + CF::kSmem);
+  uint32_t* ctrl = reinterpret_cast<uint32_t*>(bars + CF::kNumBars);   // TMEM address, home role, item, abort
+  volatile int* sh_abort = reinterpret_cast<volatile int*>(ctrl + 3);
   const int tid = threadIdx.x, warp = tid >> 5;
-
+  if (smem_u32(smem) & 1023u) {   // the swizzled tiles need 1024-byte alignment
+    if (tid == 0) record_error(p, POD_ERR_UNSUPPORTED, 1024);
+    return;
+  }
   if (tid == 0) {
-    for (int i = 0; i < 4 + kWarpsPerCta * CF::kNS; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < CF::kNumBars; ++i) {
+      uint32_t count = 1;
+      if (i == kBarSFree || i == kBarSFree + 1) count = kWarpsPerCta;
+      if (i == kBarPFull || i == kBarPFull + 1) count = kBM;
+      mbar_init(&bars[i], count);
+    }
     fence_mbar_init();
-    sh_abort = 0;
+    *sh_abort = 0;
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
     int home = p.mode == kDecodeOnly ? kRoleDecode : kRolePrefill;
@@ -528,23 +646,22 @@ __global__ void __launch_bounds__(128, 2) pod_attn_kernel(const __grid_constant_
       const int span = p.ratio_p + p.ratio_d;
       home = (span > 0 && (t % span) < p.ratio_p) ? kRolePrefill : kRoleDecode;
     }
-    sh_home = home;
+    ctrl[1] = (uint32_t)home;
   }
   __syncwarp();
   if (p.use_tmem && warp == 0) {
-    tmem_alloc(&tmem_holder, kTmemCols);
+    tmem_alloc(&ctrl[0], kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = p.use_tmem ? tmem_holder : 0u;
-  const int home = sh_home;
+  const uint32_t tmem = p.use_tmem ? ctrl[0] : 0u;
+  const int home = (int)ctrl[1];
 
-  PrefillState st{0u, {0u, 0u}, 0u};
-  uint32_t seq = 0;
-  uint8_t* ring = smem + warp * CF::kNS * CF::kDecStage;
-  uint64_t* wbars = &bars[4 + warp * CF::kNS];
+  uint32_t tiles_done = 0, items_done = 0, seq = 0;
+  uint8_t* ring = smem + (warp < kWarpsPerCta ? warp : 0) * CF::kNS * CF::kDecStage;
+  uint64_t* wbars = &bars[kBarDecode + (warp < kWarpsPerCta ? warp : 0) * CF::kNS];
 
   for (int phase = 0; phase < 2; ++phase) {
     const int role = phase == 0 ? home : 1 - home;
@@ -552,10 +669,9 @@ __global__ void __launch_bounds__(128, 2) pod_attn_kernel(const __grid_constant_
     if (p.mode == kDecodeOnly && role != kRoleDecode) continue;
     if (role == kRolePrefill) {
       while (true) {
-        if (tid == 0) sh_item = sh_abort ? p.n_pre : atomicAdd(&p.counters[kNextPrefill], 1);
+        if (tid == 0) ctrl[2] = (uint32_t)(*sh_abort ? p.n_pre : atomicAdd(&p.counters[kNextPrefill], 1));
         __syncthreads();
-        const int item = sh_item;
-        __syncthreads();
+        const int item = (int)ctrl[2];
         if (item >= p.n_pre) break;
         if (tid == 0 && p.trace) {
           int32_t* e = p.trace + 4 * item;
@@ -564,14 +680,27 @@ __global__ void __launch_bounds__(128, 2) pod_attn_kernel(const __grid_constant_
           e[2] = home;
           atomicAdd(&e[3], 1);
         }
-        if (!prefill_item<D>(p, item, smem, bars, tmem, st)) {
-          if (tid == 0) sh_abort = 1;
+        const int4 it = __ldg(&p.pre_items[item]);
+        bool ok;
+        if (warp == kMmaWarp) ok = prefill_mma<D>(p, it, smem, bars, tmem, tiles_done, items_done);
+        else if (warp == kTmaWarp) ok = prefill_tma<D>(p, it, smem, bars, tiles_done);
+        else ok = prefill_softmax<D>(p, it, smem, bars, tmem, tiles_done);
+        tc_fence_before();
+        const int fail = __syncthreads_or(!ok);
+        tc_fence_after();
+        if (fail) {
+          if (tid == 0) {
+            record_error(p, POD_ERR_TIMEOUT, 2);
+            *sh_abort = 1;
+          }
           __syncthreads();
           break;
         }
+        tiles_done += (uint32_t)((it.z + kBN - 1) / kBN);
+        items_done += 1;
       }
     } else {
-      decode_warp<D>(p, ring, wbars, seq, &sh_abort, home);
+      if (warp < kWarpsPerCta) decode_warp<D>(p, ring, wbars, seq, sh_abort, home);
       __syncthreads();
     }
   }
@@ -665,17 +794,17 @@ int launch(const pod_attn_plan_t* pl, PodParams& prm, const MergeParams& mp, cud
       prm.mode = kPrefillOnly;
       prm.use_tmem = 1;
       const int grid = pl->n_pre < pl->grid ? pl->n_pre : pl->grid;
-      pod_attn_kernel<D><<<grid, 128, smem, st>>>(prm);
+      pod_attn_kernel<D><<<grid, kThreads, smem, st>>>(prm);
     }
     if (pl->n_dec > 0) {
       prm.mode = kDecodeOnly;
       prm.use_tmem = 0;
-      pod_attn_kernel<D><<<pl->grid, 128, smem, st>>>(prm);
+      pod_attn_kernel<D><<<pl->grid, kThreads, smem, st>>>(prm);
     }
   } else if (pl->n_pre > 0 || pl->n_dec > 0) {
     prm.mode = kFused;
     prm.use_tmem = pl->n_pre > 0 ? 1 : 0;
-    pod_attn_kernel<D><<<pl->grid, 128, smem, st>>>(prm);
+    pod_attn_kernel<D><<<pl->grid, kThreads, smem, st>>>(prm);
   }
   if (pl->ev_stop) cudaEventRecord(static_cast<cudaEvent_t>(pl->ev_stop), st);
   if (pl->n_merge > 0) pod_merge_kernel<D><<<pl->n_merge, 128, 0, st>>>(mp);
