@@ -68,6 +68,8 @@ enum {
 /* config.flags */
 #define POD_FLAG_SEQUENTIAL 1u  /* ablation: prefill kernel, then decode kernel, then merge */
 #define POD_FLAG_TRACE 2u       /* record the per-item schedule into `trace` */
+#define POD_FLAG_MERGE_KERNEL 4u /* merge split-KV partials in a separate kernel after the attention
+                                   kernel(s), instead of by the last split to finish inside them */
 
 typedef struct pod_attn_config {
   int32_t num_q_heads;      /* Hq */
@@ -123,7 +125,8 @@ int pod_attn_plan_get_info(const pod_attn_plan_t* plan, pod_attn_plan_info* info
 
 /* Host copies of the work tables, for bit-exact checks; any pointer may be null.
  *   prefill_items int32 [num_prefill_items, 4]: q0, q_head, kv_end, partial (-1)
- *   decode_items  int32 [num_decode_items, 8]:  r, kv_head, k0, k1, partial (-1 = unsplit), 0, 0, 0
+ *   decode_items  int32 [num_decode_items, 8]:  r, kv_head, k0, k1, partial (-1 = unsplit),
+ *                                               merge item (-1 = unsplit), splits of the row, 0
  *   merge_items   int32 [num_merge_items, 4]:   r, kv_head, first_partial, num_splits */
 int pod_attn_plan_tables(const pod_attn_plan_t* plan, int32_t* prefill_items,
                          int32_t* decode_items, int32_t* merge_items);
@@ -135,10 +138,12 @@ int pod_attn_plan_tables(const pod_attn_plan_t* plan, int32_t* prefill_items,
  * Errors: POD_ERR_INVALID_ARG, POD_ERR_WORKSPACE, POD_ERR_CUDA. */
 int pod_attn_upload(const pod_attn_plan_t* plan, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Enqueue one hybrid-batch attention on `stream`: reset the ticket and queue
- * counters in the workspace, launch the persistent fused kernel (or, with
+/* Enqueue one hybrid-batch attention on `stream`: reset the ticket, queue and
+ * merge counters in the workspace, launch the persistent fused kernel (or, with
  * POD_FLAG_SEQUENTIAL in the plan's config, the prefill-only then decode-only
- * kernels), then the LSE merge kernel when the plan has splits.  Asynchronous.
+ * kernels).  Split-KV partials are merged by the warp that finishes a row's
+ * last split (a completion counter, no waiting), or, with POD_FLAG_MERGE_KERNEL,
+ * by the LSE merge kernel launched afterwards.  Asynchronous.
  * q/k/v/o pointers: device, 16-byte aligned; unused sides (P == 0 or B == 0)
  * may be null.  num_blocks = pages in each cache pool.  trace (nullable, used
  * with POD_FLAG_TRACE): int32 [num_prefill_items + num_decode_items, 4], zeroed

@@ -24,10 +24,11 @@ Rule
     S_r = ceil(pages_r / c) splits; split s covers pages
     [floor(s pages_r / S_r), floor((s+1) pages_r / S_r)), i.e. tokens
     [16 p0, min(16 p1, L_r)).
-  Decode items (r, kv_head, k0, k1, partial, 0, 0, 0): partial = running index
-    over (r, kv_head, s) of rows with S_r > 1, else -1; sorted by
-    (-pages, r, kv_head, s).
-  Merge items (r, kv_head, first_partial, S_r) for every (r, kv_head) with S_r > 1.
+  Decode items (r, kv_head, k0, k1, partial, merge, S_r, 0): partial = running
+    index over (r, kv_head, s) of rows with S_r > 1, else -1; merge = index of
+    the row's merge item, else -1; sorted by (-pages, r, kv_head, s).
+  Merge items (r, kv_head, first_partial, S_r) for every (r, kv_head) with S_r > 1,
+    in (r, kv_head) order.
   Ratio p:d of per-SM tickets (ticket t -> prefill iff t mod (p+d) < p):
     explicit (ratio_p, ratio_d) reduced by gcd (a zero side gives 1:0 or 0:1);
     proportional (both 0): no prefill -> 0:1; no decode -> 1:0; otherwise
@@ -122,6 +123,7 @@ def plan_ref(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
         S = _ceil(pages[r], c) if pages[r] > 0 else 1
         for kvh in range(Hkv):
             first = npart
+            midx = len(merge) if S > 1 else -1
             for s in range(S):
                 p0 = (s * pages[r]) // S
                 p1 = ((s + 1) * pages[r]) // S
@@ -129,7 +131,7 @@ def plan_ref(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
                 if S > 1:
                     part = npart
                     npart += 1
-                dec.append((p1 - p0, r, kvh, s, (r, kvh, PAGE * p0, min(PAGE * p1, lens[r]), part, 0, 0, 0)))
+                dec.append((p1 - p0, r, kvh, s, (r, kvh, PAGE * p0, min(PAGE * p1, lens[r]), part, midx, S, 0)))
             if S > 1:
                 merge.append((r, kvh, first, S))
     dec.sort(key=lambda e: (-e[0], e[1], e[2], e[3]))

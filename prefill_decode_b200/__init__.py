@@ -27,6 +27,7 @@ POD_ERR_TIMEOUT = -6
 POD_ERR_PLAN_MISMATCH = -7
 POD_FLAG_SEQUENTIAL = 1
 POD_FLAG_TRACE = 2
+POD_FLAG_MERGE_KERNEL = 4
 
 EXPORTED = [
     "pod_attn_plan", "pod_attn_plan_get_info", "pod_attn_plan_tables", "pod_attn_upload", "pod_attn_run",

@@ -98,12 +98,13 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t k
     const int32_t S = (int32_t)ceil_div(pages[r], c);
     for (int32_t kvh = 0; kvh < Hkv; ++kvh) {
       const int32_t first = npart;
+      const int32_t midx = S > 1 ? (int32_t)(pl->merge.size() / kMergeItemInts) : -1;
       for (int32_t s = 0; s < S; ++s) {
         const int32_t p0 = (int32_t)(((int64_t)s * pages[r]) / S);
         const int32_t p1 = (int32_t)(((int64_t)(s + 1) * pages[r]) / S);
         int32_t part = -1;
         if (S > 1) part = npart++;
-        DecEntry e{p1 - p0, r, kvh, s, {r, kvh, kPage * p0, std::min(kPage * p1, lens[r]), part, 0, 0, 0}};
+        DecEntry e{p1 - p0, r, kvh, s, {r, kvh, kPage * p0, std::min(kPage * p1, lens[r]), part, midx, S, 0}};
         ents.push_back(e);
       }
       if (S > 1) {
@@ -171,7 +172,8 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t k
   pl->ratio_d = rd;
 
   // ---- workspace layout and the host image of the tables
-  pl->off_pre = kCountersBytes;
+  pl->off_merge_cnt = kCountersBytes;
+  pl->off_pre = align_up(pl->off_merge_cnt + 4LL * pl->n_merge, 256);
   pl->off_dec = align_up(pl->off_pre + 4LL * kPrefillItemInts * pl->n_pre, 256);
   pl->off_merge = align_up(pl->off_dec + 4LL * kDecodeItemInts * pl->n_dec, 256);
   pl->off_part_o = align_up(pl->off_merge + 4LL * kMergeItemInts * pl->n_merge, 256);

@@ -52,6 +52,8 @@ struct alignas(64) PodParams {
   int32_t* counters;
   const int4* pre_items;
   const int4* dec_items;   // two int4 per item
+  const int4* merge_items; // r, kvh, first_partial, num_splits
+  int32_t* merge_cnt;      // splits finished per merge item (zero at launch)
   float* part_o;
   float* part_lse;
   int32_t* trace;
@@ -63,6 +65,7 @@ struct alignas(64) PodParams {
   int32_t ratio_p, ratio_d;
   int32_t mode;
   int32_t use_tmem;
+  int32_t merge_in_kernel; // 1: the warp finishing a row's last split merges the row
   float scale_log2;        // softmax scale * log2(e)
 };
 
@@ -72,17 +75,25 @@ constexpr int kTmaWarp = 5;
 
 // mbarrier slots in the CTA control block
 enum : int {
-  kBarQ = 0,        // Q tile landed (TMA)                                    count 1 + tx
-  kBarKFull = 1,    // [3] K tile landed (TMA)                                count 1 + tx
-  kBarKEmpty = 4,   // [3] K slot free again: its P.V finished (MMA commit)   count 1
-  kBarVFull = 7,    // [2] V tile landed (TMA)                                count 1 + tx
-  kBarVEmpty = 9,   // [2] V slot free again (MMA commit)                     count 1
-  kBarSFull = 11,   // [2] S tile ready in TMEM (MMA commit)                  count 1
-  kBarSFree = 13,   // [2] S tile read out by the 4 softmax warps             count 4
-  kBarPFull = 15,   // [2] P tile written (and O rescaled) by 128 rows        count 128
-  kBarODone = 17,   // P.V MMA of a tile finished (MMA commit)                count 1
-  kBarDecode = 18,  // [kWarpsPerCta * kNS] decode page rings                 count 1 + tx
+  kBarQ = 0,        // Q tile landed (TMA)                                      count 1 + tx
+  kBarKFull = 1,    // [3] K tile landed (TMA)                                  count 1 + tx
+  kBarKEmpty = 4,   // [3] K slot free again: its S MMA finished (commit)       count 1
+  kBarVFull = 7,    // [2] V tile landed (TMA)                                  count 1 + tx
+  kBarVEmpty = 9,   // [2] V slot free again: its P.V MMA finished (commit)     count 1
+  kBarSFull = 11,   // [2] S tile ready in TMEM buffer t&1 (commit)             count 1
+  kBarPFull = 13,   // [2] P tile stored over S in TMEM (and O rescaled)        count 4 (softmax warps)
+  kBarODone = 15,   // [2] P.V MMA of tile t finished, slot t&1 (commit)        count 1
+  kBarOFinal = 17,  // last P.V MMA of an item finished (commit)                count 1
+  kBarDecode = 18,  // [kWarpsPerCta * kNS] decode page rings                   count 1 + tx
 };
+// Parity waits are only sound when the waiter knows the barrier is at most one
+// phase away from the one it waits for.  For key tile t (counted over the
+// CTA's lifetime): S_t goes into TMEM buffer t&1 only after P.V of tile t-2
+// (which read P_{t-2} from that buffer) finished, and P.V_t needs P_t, so
+// s_full, p_full and o_done can never run two phases ahead of their waiters;
+// the softmax waits for P.V of tile t-1 on o_done[(t-1)&1], whose previous
+// phase (tile t-3) finished before S_t was issued; the epilogue waits on
+// o_final, which completes once per item.
 
 template <int D>
 struct Cfg {
@@ -91,12 +102,9 @@ struct Cfg {
   static constexpr int kKTile = kBN * D * 2;                  // 64 keys of K (or V)
   static constexpr int kKSlots = 3;                           // K ring: two tiles of lead
   static constexpr int kVSlots = 2;                           // V ring: two tiles of lead
-  static constexpr int kPBytes = kBM * kBN * 2;               // P tile [128 x 64] bf16
-  static constexpr bool kPAliasK = (kPBytes <= kKTile);       // P is written over its spent K tile
   static constexpr int kOffK = kQBytes;
   static constexpr int kOffV = kOffK + kKSlots * kKTile;
-  static constexpr int kOffP = kOffV + kVSlots * kKTile;
-  static constexpr int kPrefillSmem = kOffP + (kPAliasK ? 0 : 2 * kPBytes);
+  static constexpr int kPrefillSmem = kOffV + kVSlots * kKTile;
   static constexpr int kPageBytes = kPage * D * 2;            // one 16-token page of one kv head
   static constexpr int kDecStage = 2 * kPageBytes;            // K page + V page
   static constexpr int kNS = (kPrefillSmem / kWarpsPerCta) / kDecStage;   // decode ring depth per warp
@@ -133,9 +141,6 @@ struct PrefillSmem {
   __device__ uint8_t* q() const { return base; }
   __device__ uint8_t* k(uint32_t t) const { return base + Cfg<D>::kOffK + (t % Cfg<D>::kKSlots) * Cfg<D>::kKTile; }
   __device__ uint8_t* v(uint32_t t) const { return base + Cfg<D>::kOffV + (t % Cfg<D>::kVSlots) * Cfg<D>::kKTile; }
-  __device__ uint8_t* pt(uint32_t t) const {
-    return Cfg<D>::kPAliasK ? k(t) : base + Cfg<D>::kOffP + (t & 1u) * Cfg<D>::kPBytes;
-  }
 };
 
 // TMA warp: tensor-map rows of the 4 pages of key tile kb (lanes 0..3 look the
@@ -194,19 +199,20 @@ __device__ bool prefill_tma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
     const bool more_k = j + CF::kKSlots < nkb;
     const int rk = more_k ? tile_page_row(p, j + CF::kKSlots, kvh, kv_end, lane) : 0;
     const int rv = tile_page_row(p, j + CF::kVSlots, kvh, kv_end, lane);
-    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarVEmpty + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs))) return false;
-    issue_tile<D>(&p.tm_v, sm.v(t + CF::kVSlots), &bars[kBarVFull + (t & 1u)], rv, lane);
-    if (more_k) {
+    if (more_k) {                // K first: the MMA warp needs it two tiles ahead
       if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKEmpty + t % 3], (t / 3) & 1u, kWaitLimitNs))) return false;
       issue_tile<D>(&p.tm_k, sm.k(t + CF::kKSlots), &bars[kBarKFull + t % 3], rk, lane);
     }
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarVEmpty + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs))) return false;
+    issue_tile<D>(&p.tm_v, sm.v(t + CF::kVSlots), &bars[kBarVFull + (t & 1u)], rv, lane);
   }
   return true;
 }
 
 // MMA warp of one prefill item (lane 0 issues): S_t = Q K_t^T into TMEM buffer
-// t&1 one tile ahead of the softmax; O += P_t V_t once P_t is written; each
-// P.V commit frees the tile's K and V slots and signals O.
+// t&1, two tiles ahead of the softmax; O += P_t V_t with P_t read from TMEM
+// (stored by the softmax over the first 32 columns of S_t).  Commits free the
+// K slot right after S_t and the V slot and the TMEM buffer after P.V_t.
 template <int D>
 __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t tmem, uint32_t t0,
                             uint32_t nq) {
@@ -221,7 +227,6 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
   const uint64_t dq = sdesc_sw128(smem_u32(sm.q()), 16, 1024);
   const uint64_t dk0 = sdesc_sw128(smem_u32(smem + CF::kOffK), 16, 1024);
   const uint64_t dv0 = sdesc_sw128(smem_u32(smem + CF::kOffV), kBN * 128, 1024);
-  const uint64_t dp0 = sdesc_sw128(smem_u32(CF::kPAliasK ? smem + CF::kOffK : smem + CF::kOffP), 16, 1024);
 
   auto issue_s = [&](uint32_t t) {
     const uint64_t dk = dk0 + (uint64_t)(((t % CF::kKSlots) * CF::kKTile) >> 4);
@@ -232,32 +237,23 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
       umma_bf16(tmem + (t & 1u) * kBN, dq + aoff, dk + boff, idesc_s, kk > 0 ? 1u : 0u);
     }
     umma_commit(&bars[kBarSFull + (t & 1u)]);
+    umma_commit(&bars[kBarKEmpty + t % 3]);
   };
 
-  bool w = mbar_wait(&bars[kBarQ], nq & 1u, kWaitLimitNs) &&
-           mbar_wait(&bars[kBarKFull + t0 % 3], (t0 / 3) & 1u, kWaitLimitNs);
-  if (t0 >= 2) w = w && mbar_wait(&bars[kBarSFree + (t0 & 1u)], ((t0 - 2) >> 1) & 1u, kWaitLimitNs);
-  if (!__all_sync(0xffffffffu, w)) return false;
-  if (lane == 0) {
-    tc_fence_after();
-    issue_s(t0);
+  if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarQ], nq & 1u, kWaitLimitNs))) return false;
+  for (int i = 0; i < 2 && i < nkb; ++i) {   // S of the first two tiles
+    const uint32_t tn = t0 + i;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + tn % 3], (tn / 3) & 1u, kWaitLimitNs))) return false;
+    if (lane == 0) {
+      tc_fence_after();
+      issue_s(tn);
+    }
+    __syncwarp();
   }
-  __syncwarp();
   for (int j = 0; j < nkb; ++j) {
     const uint32_t t = t0 + j;
-    if (j + 1 < nkb) {           // S of the next tile runs while the softmax works on this one
-      const uint32_t tn = t + 1;
-      bool ws = mbar_wait(&bars[kBarKFull + tn % 3], (tn / 3) & 1u, kWaitLimitNs);
-      if (tn >= 2) ws = ws && mbar_wait(&bars[kBarSFree + (tn & 1u)], ((tn - 2) >> 1) & 1u, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, ws)) return false;
-      if (lane == 0) {
-        tc_fence_after();
-        issue_s(tn);
-      }
-      __syncwarp();
-    }
-    bool wp = mbar_wait(&bars[kBarVFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs) &&
-              mbar_wait(&bars[kBarPFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs);
+    const bool wp = mbar_wait(&bars[kBarVFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs) &&
+                    mbar_wait(&bars[kBarPFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs);
     if (!__all_sync(0xffffffffu, wp)) return false;
     const int valid = kv_end - j * kBN;
     if (valid < kBN) {           // V rows past the request's end may hold anything: zero them
@@ -272,17 +268,28 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
     }
     if (lane == 0) {
       tc_fence_after();
-      const uint64_t dp = dp0 + (uint64_t)((CF::kPAliasK ? (t % CF::kKSlots) * CF::kKTile : (t & 1u) * CF::kPBytes) >> 4);
       const uint64_t dv = dv0 + (uint64_t)(((t & 1u) * CF::kKTile) >> 4);
+      const uint32_t pa = tmem + (t & 1u) * kBN;
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk)
-        umma_bf16(tmem + kTmemO, dp + (uint64_t)((kk * 32) >> 4), dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_o,
-                  (j > 0 || kk > 0) ? 1u : 0u);
-      umma_commit(&bars[kBarODone]);
-      umma_commit(&bars[kBarKEmpty + t % 3]);
+        umma_bf16_tmem_a(tmem + kTmemO, pa + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_o,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(&bars[kBarODone + (t & 1u)]);
       umma_commit(&bars[kBarVEmpty + (t & 1u)]);
+      if (j == nkb - 1) umma_commit(&bars[kBarOFinal]);
     }
     __syncwarp();
+    if (j + 2 < nkb) {           // S_{t+2} into buffer t&1 once P.V_t has read P_t from it
+      const uint32_t tn = t + 2;
+      const bool ws = mbar_wait(&bars[kBarODone + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs) &&
+                      mbar_wait(&bars[kBarKFull + tn % 3], (tn / 3) & 1u, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ws)) return false;
+      if (lane == 0) {
+        tc_fence_after();
+        issue_s(tn);
+      }
+      __syncwarp();
+    }
   }
   return true;
 }
@@ -294,11 +301,10 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
 // K-major 128B-swizzled layout; finally O / l -> bf16 -> global.
 template <int D>
 __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t tmem,
-                                uint32_t t0) {
+                                uint32_t t0, uint32_t nq) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q0 = it.x, qh = it.y, kv_end = it.z;
   const int nkb = (kv_end + kBN - 1) / kBN;
-  const PrefillSmem<D> sm{smem};
   const int row = tid;
   const int row_limit = min(p.C + q0 + row + 1, kv_end);
   const int full_tiles = (p.C + q0 + 1) / kBN;   // tiles visible to every row of this item
@@ -313,31 +319,28 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
     tmem_ld32(tmem + t_lane + (t & 1u) * kBN, s);
     tmem_ld32(tmem + t_lane + (t & 1u) * kBN + 32, s + 32);
     tmem_wait_ld();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars[kBarSFree + (t & 1u)]);
-    float mx = -INFINITY;
+    float mx = -INFINITY;        // row max of the raw scores; m below is in scaled (log2) units
     if (j < full_tiles) {
 #pragma unroll
-      for (int k = 0; k < kBN; ++k) {
-        s[k] *= sl2;
-        mx = fmaxf(mx, s[k]);
-      }
+      for (int k = 0; k < kBN; ++k) mx = fmaxf(mx, s[k]);
     } else {
       const int lim = row_limit - j * kBN;
 #pragma unroll
       for (int k = 0; k < kBN; ++k) {
-        s[k] = k < lim ? s[k] * sl2 : -INFINITY;
+        s[k] = k < lim ? s[k] : -INFINITY;
         mx = fmaxf(mx, s[k]);
       }
     }
+    mx *= sl2;
     if (j == 0) {
       m = mx;
     } else {
       const bool need = mx > m + 8.f;
       if (__any_sync(0xffffffffu, need)) {
         // O holds the P.V sums of the earlier tiles: wait for the last one, then rescale
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone], (t - 1) & 1u, kWaitLimitNs))) return false;
+        const uint32_t tp = t - 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone + (tp & 1u)], (tp >> 1) & 1u, kWaitLimitNs)))
+          return false;
         tc_fence_after();
         const float m_new = need ? mx : m;
         const float alpha = ex2(m - m_new);
@@ -356,30 +359,25 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
       }
     }
     float rs = 0.f;
-    uint8_t* prow = sm.pt(t) + row * 128;
+    const float neg_m = -m;
+    uint32_t pk[kBN / 2];
 #pragma unroll
-    for (int c = 0; c < kBN / 8; ++c) {
-      float e[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        e[k] = ex2(s[c * 8 + k] - m);
-        rs += e[k];
-      }
-      uint4 v;
-      v.x = pack_bf16(e[0], e[1]);
-      v.y = pack_bf16(e[2], e[3]);
-      v.z = pack_bf16(e[4], e[5]);
-      v.w = pack_bf16(e[6], e[7]);
-      *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v;
+    for (int k = 0; k < kBN / 2; ++k) {
+      const float e0 = ex2(fmaf(s[2 * k], sl2, neg_m));
+      const float e1 = ex2(fmaf(s[2 * k + 1], sl2, neg_m));
+      rs += e0 + e1;
+      pk[k] = pack_bf16(e0, e1);
     }
     l += rs;
-    fence_proxy_async_smem();
+    // P_t (bf16 pairs) over the first 32 columns of S_t: the A operand of P.V_t
+    tmem_st32_u(tmem + t_lane + (t & 1u) * kBN, pk);
+    tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(&bars[kBarPFull + (t & 1u)]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[kBarPFull + (t & 1u)]);
   }
   // epilogue: O / l -> bf16, one 2*D-byte row per thread
-  const uint32_t tl = t0 + nkb - 1;
-  if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone], tl & 1u, kWaitLimitNs))) return false;
+  if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarOFinal], nq & 1u, kWaitLimitNs))) return false;
   tc_fence_after();
   const int q = q0 + row;
   const float inv = 1.f / l;
@@ -432,6 +430,36 @@ __device__ __forceinline__ uint32_t swz(int row, int col_elem) {
   return (uint32_t)(row * 128 + ((((col_elem >> 3) ^ row) & 7) << 4));
 }
 
+// One warp merges the split partials of merge item `midx` into bf16 outputs:
+// O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s (log2 domain).
+// The partials were written by other warps of this launch: read them through L2.
+template <int D>
+__device__ void merge_row_warp(const PodParams& p, int midx) {
+  const int lane = threadIdx.x & 31;
+  const int4 mi = __ldg(&p.merge_items[midx]);
+  const int r = mi.x, kvh = mi.y, first = mi.z, S = mi.w;
+  const int g = p.g;
+  for (int h = 0; h < g; ++h) {
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(&p.part_lse[(size_t)(first + s) * g + h]));
+    float acc[D / 32];
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
+    float den = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float w = ex2(__ldcg(&p.part_lse[(size_t)(first + s) * g + h]) - M);
+      den += w;
+      const float* po = p.part_o + ((size_t)(first + s) * g + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) acc[c] += w * __ldcg(&po[lane + 32 * c]);
+    }
+    const float inv = 1.f / den;
+    __nv_bfloat16* ob = p.o_dec + ((size_t)r * p.Hq + kvh * g + h) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) ob[lane + 32 * c] = __float2bfloat16_rn(acc[c] * inv);
+  }
+}
+
 template <int D>
 __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, uint32_t& seq,
                             volatile int* abort_flag, int home_role) {
@@ -446,7 +474,7 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
     if (item >= p.n_dec) return true;
     const int4 a = __ldg(&p.dec_items[2 * item]);
     const int4 b = __ldg(&p.dec_items[2 * item + 1]);
-    const int r = a.x, kvh = a.y, k0 = a.z, k1 = a.w, part = b.x;
+    const int r = a.x, kvh = a.y, k0 = a.z, k1 = a.w, part = b.x, midx = b.y, nsplit = b.z;
     const int p0 = k0 / kPage;
     const int np = (k1 - k0 + kPage - 1) / kPage;
     if (lane == 0) {
@@ -608,6 +636,18 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         if (hA < g) p.part_lse[(size_t)part * g + hA] = mA + __log2f(lA);
         if (hB < g) p.part_lse[(size_t)part * g + hB] = mB + __log2f(lB);
       }
+      if (p.merge_in_kernel) {
+        // the warp that finishes a row's last split merges it (no waiting on other warps)
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = atomicAdd(&p.merge_cnt[midx], 1) == nsplit - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          merge_row_warp<D>(p, midx);
+        }
+      }
     }
   }
 }
@@ -631,8 +671,7 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
   if (tid == 0) {
     for (int i = 0; i < CF::kNumBars; ++i) {
       uint32_t count = 1;
-      if (i == kBarSFree || i == kBarSFree + 1) count = kWarpsPerCta;
-      if (i == kBarPFull || i == kBarPFull + 1) count = kBM;
+      if (i == kBarPFull || i == kBarPFull + 1) count = kWarpsPerCta;
       mbar_init(&bars[i], count);
     }
     fence_mbar_init();
@@ -684,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
         bool ok;
         if (warp == kMmaWarp) ok = prefill_mma<D>(p, it, smem, bars, tmem, tiles_done, items_done);
         else if (warp == kTmaWarp) ok = prefill_tma<D>(p, it, smem, bars, tiles_done);
-        else ok = prefill_softmax<D>(p, it, smem, bars, tmem, tiles_done);
+        else ok = prefill_softmax<D>(p, it, smem, bars, tmem, tiles_done, items_done);
         tc_fence_before();
         const int fail = __syncthreads_or(!ok);
         tc_fence_after();
@@ -807,7 +846,8 @@ int launch(const pod_attn_plan_t* pl, PodParams& prm, const MergeParams& mp, cud
     pod_attn_kernel<D><<<pl->grid, kThreads, smem, st>>>(prm);
   }
   if (pl->ev_stop) cudaEventRecord(static_cast<cudaEvent_t>(pl->ev_stop), st);
-  if (pl->n_merge > 0) pod_merge_kernel<D><<<pl->n_merge, 128, 0, st>>>(mp);
+  if (pl->n_merge > 0 && (pl->cfg.flags & POD_FLAG_MERGE_KERNEL))
+    pod_merge_kernel<D><<<pl->n_merge, 128, 0, st>>>(mp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return POD_OK;
@@ -888,7 +928,7 @@ int pod_attn_upload(const pod_attn_plan_t* pl, void* ws, size_t ws_bytes, void* 
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return POD_ERR_INVALID_ARG;
   if ((int64_t)ws_bytes < pl->ws_bytes) return POD_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(ws, 0, kCountersBytes, st);
+  cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)pl->off_pre, st);
   if (e == cudaSuccess && !pl->image.empty())
     e = cudaMemcpyAsync(static_cast<uint8_t*>(ws) + kCountersBytes, pl->image.data(), pl->image.size(),
                         cudaMemcpyHostToDevice, st);
@@ -955,6 +995,9 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   prm.counters = reinterpret_cast<int32_t*>(w);
   prm.pre_items = reinterpret_cast<const int4*>(w + pl->off_pre);
   prm.dec_items = reinterpret_cast<const int4*>(w + pl->off_dec);
+  prm.merge_items = reinterpret_cast<const int4*>(w + pl->off_merge);
+  prm.merge_cnt = reinterpret_cast<int32_t*>(w + pl->off_merge_cnt);
+  prm.merge_in_kernel = (pl->cfg.flags & POD_FLAG_MERGE_KERNEL) ? 0 : 1;
   prm.part_o = reinterpret_cast<float*>(w + pl->off_part_o);
   prm.part_lse = reinterpret_cast<float*>(w + pl->off_part_lse);
   prm.trace = (pl->cfg.flags & POD_FLAG_TRACE) ? trace : nullptr;
@@ -982,8 +1025,8 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   mp.Hq = Hq;
   mp.g = pl->g;
 
-  // counters (tickets, queue heads, error word) start at zero every run
-  cudaError_t e = cudaMemsetAsync(ws, 0, kCountersBytes, st);
+  // counters (tickets, queue heads, error word, merge completions) start at zero every run
+  cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)pl->off_pre, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return D == 128 ? launch<128>(pl, prm, mp, st) : launch<64>(pl, prm, mp, st);
 }

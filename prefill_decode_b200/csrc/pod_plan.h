@@ -16,7 +16,8 @@ constexpr int kWarpsPerCta = 4;      // 128-thread CTAs; 4 single-warp decode un
 constexpr int kMaxSms = 512;         // ticket slots (smid is folded modulo this)
 constexpr int kCostRatio = 248;      // B200 tensor FLOP/s per HBM byte/s (1624.7e12 / 6539.5e9)
 
-// Workspace layout (bytes).  Counters first; the tables follow in the order
+// Workspace layout (bytes).  Counters first, then one completion counter per
+// merge item (both zeroed every run); the tables follow in the order
 // prefill items | decode items | merge items; then split partials.
 constexpr int64_t kCountersBytes = 4096;
 constexpr int kTicketBase = 0;       // int32 [kMaxSms]
@@ -25,7 +26,7 @@ constexpr int kNextDecode = 513;     // int32
 constexpr int kErrorWord = 514;      // int32 (first error code recorded)
 constexpr int kErrorInfo = 515;      // int32 (item or block that caused it)
 constexpr int kPrefillItemInts = 4;  // q0, q_head, kv_end, partial
-constexpr int kDecodeItemInts = 8;   // r, kv_head, k0, k1, partial, 0, 0, 0
+constexpr int kDecodeItemInts = 8;   // r, kv_head, k0, k1, partial, merge item, splits, 0
 constexpr int kMergeItemInts = 4;    // r, kv_head, first_partial, num_splits
 
 inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -37,6 +38,7 @@ struct pod_attn_plan {
   int32_t P = 0, C = 0, B = 0, g = 1;
   int32_t n_pre = 0, n_dec = 0, n_merge = 0, n_part = 0;
   int32_t ctas = 2, ratio_p = 1, ratio_d = 1, chunk_pages = 16, num_sms = 148, grid = 0;
+  int64_t off_merge_cnt = 0;   // int32 per merge item: splits finished (reset to 0 by the merging warp)
   int64_t off_pre = 0, off_dec = 0, off_merge = 0, off_part_o = 0, off_part_lse = 0, ws_bytes = 0;
   int64_t prefill_flops = 0, decode_flops = 0, kv_bytes = 0, qo_bytes = 0;
   std::vector<int32_t> decode_lens;

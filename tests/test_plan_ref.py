@@ -41,8 +41,14 @@ def check_plan(pl, Hq, Hkv, P, C, lens, sms=SMS, waves=2, minc=16):
     assert q0s == sorted(q0s, reverse=True)
     # decode coverage: every key of every (r, kvh) exactly once, page-aligned splits
     cover = {}
-    for r, kvh, k0, k1, part, a, b, c in pl.decode_items.tolist():
-        assert a == b == c == 0
+    merges = pl.merge_items.tolist()
+    for r, kvh, k0, k1, part, midx, nsplit, c in pl.decode_items.tolist():
+        assert c == 0
+        if part < 0:
+            assert midx == -1 and nsplit == 1
+        else:
+            assert merges[midx][:2] == [r, kvh] and merges[midx][3] == nsplit
+            assert merges[midx][2] <= part < merges[midx][2] + nsplit
         assert 0 <= r < len(lens) and 0 <= kvh < Hkv
         assert k0 % PAGE == 0 and k0 < k1 <= lens[r]
         assert (k1 - k0) <= pl.chunk_pages * PAGE or part == -1
