@@ -432,31 +432,63 @@ __device__ __forceinline__ uint32_t swz(int row, int col_elem) {
 
 // One warp merges the split partials of merge item `midx` into bf16 outputs:
 // O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s (log2 domain).
-// The partials were written by other warps of this launch: read them through L2.
+// Lane l owns d elements [4l, 4l + 4) (and +128 ... for larger d) of every head,
+// so each split costs one independent 16-byte load per head and lane.  The
+// partials were written by other warps of this launch: read them through L2.
 template <int D>
 __device__ void merge_row_warp(const PodParams& p, int midx) {
+  constexpr int kV = D / 128 > 0 ? D / 128 : 1;   // float4 chunks per lane and head
   const int lane = threadIdx.x & 31;
   const int4 mi = __ldg(&p.merge_items[midx]);
   const int r = mi.x, kvh = mi.y, first = mi.z, S = mi.w;
   const int g = p.g;
-  for (int h = 0; h < g; ++h) {
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(&p.part_lse[(size_t)(first + s) * g + h]));
-    float acc[D / 32];
+  const bool active = (lane * 4) < D;
+  float M[8], den[8];
+  float4 acc[8][kV];
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
-    float den = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float w = ex2(__ldcg(&p.part_lse[(size_t)(first + s) * g + h]) - M);
-      den += w;
-      const float* po = p.part_o + ((size_t)(first + s) * g + h) * D;
+  for (int h = 0; h < 8; ++h) {
+    M[h] = -INFINITY;
+    den[h] = 0.f;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) acc[c] += w * __ldcg(&po[lane + 32 * c]);
+    for (int v = 0; v < kV; ++v) acc[h][v] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int s = 0; s < S; ++s)
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+      if (h < g) M[h] = fmaxf(M[h], __ldcg(&p.part_lse[(size_t)(first + s) * g + h]));
+  for (int s = 0; s < S; ++s) {
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      if (h < g) {
+        const float w = ex2(__ldcg(&p.part_lse[(size_t)(first + s) * g + h]) - M[h]);
+        den[h] += w;
+        const float4* po = reinterpret_cast<const float4*>(p.part_o + ((size_t)(first + s) * g + h) * D);
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+          if (active) {
+            const float4 x = __ldcg(&po[lane + 32 * v]);
+            acc[h][v].x += w * x.x;
+            acc[h][v].y += w * x.y;
+            acc[h][v].z += w * x.z;
+            acc[h][v].w += w * x.w;
+          }
+        }
+      }
     }
-    const float inv = 1.f / den;
-    __nv_bfloat16* ob = p.o_dec + ((size_t)r * p.Hq + kvh * g + h) * D;
+  }
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) ob[lane + 32 * c] = __float2bfloat16_rn(acc[c] * inv);
+  for (int h = 0; h < 8; ++h) {
+    if (h < g && active) {
+      const float inv = 1.f / den[h];
+      __nv_bfloat16* ob = p.o_dec + ((size_t)r * p.Hq + kvh * g + h) * D;
+#pragma unroll
+      for (int v = 0; v < kV; ++v) {
+        uint2 o;
+        o.x = pack_bf16(acc[h][v].x * inv, acc[h][v].y * inv);
+        o.y = pack_bf16(acc[h][v].z * inv, acc[h][v].w * inv);
+        *reinterpret_cast<uint2*>(ob + 4 * (lane + 32 * v)) = o;
+      }
+    }
   }
 }
 
@@ -688,8 +720,11 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
     ctrl[1] = (uint32_t)home;
   }
   __syncwarp();
-  if (p.use_tmem && warp == 0) {
-    tmem_alloc(&ctrl[0], kTmemCols);
+  if (warp == 0) {
+    if (p.use_tmem) tmem_alloc(&ctrl[0], kTmemCols);
+    // every CTA gives up its TMEM allocation permit at once, whether it allocated
+    // or not: a resident CTA still holding the permit keeps the SM from taking
+    // the second CTA of this kernel
     tmem_relinquish();
   }
   tc_fence_before();
@@ -817,6 +852,10 @@ int configure_kernels() {
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 64 && done[dev]) return POD_OK;
   e = cudaFuncSetAttribute(pod_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemAlloc);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // two CTAs of ~113 KB need the whole 228 KB shared-memory carveout on every launch
+  e = cudaFuncSetAttribute(pod_attn_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 64) done[dev] = true;
   return POD_OK;
