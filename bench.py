@@ -142,6 +142,27 @@ class ClockSampler:
                 "power_w_max": max((num(p[3]) or 0.0) for p in inside)}
 
 
+# ------------------------------------------------------------ multi-rank
+def reduce_max(x: float, dist, device) -> float:
+    """Max of a per-rank scalar over all ranks (timings are reported as the
+    slowest replica); identity without a process group."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def plan_digest(plan) -> str:
+    """Hash of a plan's work tables: every replica must plan its batch alike."""
+    pre, dec, mer = plan.tables()
+    h = hashlib.sha256()
+    for a in (pre, dec, mer):
+        h.update(np.ascontiguousarray(a).tobytes())
+    return h.hexdigest()[:16]
+
+
 # ---------------------------------------------------------------- CPU oracle
 def cpu_oracle_time(b, decode_reqs, prefill_rows):
     """Time the float64 oracle on a subset; return (seconds, decode part, prefill part, outputs)."""
@@ -218,6 +239,59 @@ def config_dict(w, b, mode):
             "l2": "no flush: inputs larger than L2 (the KV streamed per step exceeds 126 MB)"}
 
 
+# ---------------------------------------------------------------- sweep mode
+def run_sweep(args):
+    """Every named workload and every mix-sweep point (fused and sequential),
+    one JSON object per line; for the committed result tables, not the bench
+    line the contract reads."""
+    import torch
+    from prefill_decode_b200 import build
+    build.build()
+    import prefill_decode_b200 as pod
+    from tests.podrun import DeviceBatch
+    peaks, peak_src = load_peaks()
+    names = args.sweep.split(",") if args.sweep not in ("1", "all") else None
+    wls = [synth.NAMED[n]() for n in sorted(synth.NAMED)] + synth.sweep_points()
+    if names:
+        wls = [w for w in wls if w.name in names]
+    stream = torch.cuda.current_stream()
+    for w in wls:
+        db = DeviceBatch.generated_on_device(torch, w)
+        res = {"workload": w.name, "values": "torch.Generator(cuda, seed) normals; layout from synth"}
+        for mode, flags in (("fused", 0), ("sequential", pod.POD_FLAG_SEQUENTIAL)):
+            pl = db.plan(pod, flags=flags)
+            ws = db.workspace(pl)
+            pl.upload(ws, stream)
+            ev = [(pod.Event(), pod.Event()) for _ in range(args.steps)]
+            for _ in range(args.warmup):
+                db.run(pod, pl, ws, stream=stream)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(args.steps):
+                pl.set_events(ev[i][0].handle, ev[i][1].handle)
+                db.run(pod, pl, ws, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            pl.set_events(None, None)
+            info = pl.info
+            step_us = e0.elapsed_time(e1) * 1e3 / args.steps
+            kern_us = float(np.mean([a.elapsed_ms(c) for a, c in ev])) * 1e3
+            t_hbm = (info.kv_bytes + info.qo_bytes) / (peaks["hbm_gbs"] * 1e9) * 1e6
+            t_tc = info.prefill_flops / (peaks["bf16_tflops"] * 1e12) * 1e6
+            res[mode] = {"step_us": step_us, "kernel_us": kern_us, "roofline_us": max(t_hbm, t_tc),
+                         "frac_step": max(t_hbm, t_tc) / step_us, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                         "hbm_GBps": (info.kv_bytes + info.qo_bytes) / (kern_us * 1e-6) / 1e9,
+                         "prefill_TFLOPs": info.prefill_flops / (kern_us * 1e-6) / 1e12,
+                         "error_word": db.error_word(pl, ws)}
+        res["speedup_vs_sequential"] = res["sequential"]["step_us"] / res["fused"]["step_us"]
+        res["peaks"] = peak_src
+        print(json.dumps(res), flush=True)
+        del db
+        torch.cuda.empty_cache()
+    return 0
+
+
 # --------------------------------------------------------------------- ours
 def main():
     ap = argparse.ArgumentParser()
@@ -229,8 +303,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--sweep", default=None,
+                    help="'all' or comma-separated workload names: per-workload table lines instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.sweep:
+        args.steps = min(args.steps, 200)
+        return run_sweep(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -291,11 +370,7 @@ def main():
         return total_ms, kern, (t_wall0, t_wall1)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, dist if world > 1 else None, dev)
 
     gpu_id = str(local)
     try:

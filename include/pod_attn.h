@@ -70,6 +70,9 @@ enum {
 #define POD_FLAG_TRACE 2u       /* record the per-item schedule into `trace` */
 #define POD_FLAG_MERGE_KERNEL 4u /* merge split-KV partials in a separate kernel after the attention
                                    kernel(s), instead of by the last split to finish inside them */
+#define POD_FLAG_SELFTEST_TIMEOUT 8u /* diagnostic: CTA 0 first waits (1 ms limit) on a barrier that
+                                       nothing arrives at, so the wait expires and POD_ERR_TIMEOUT is
+                                       recorded in the error word; the attention itself still runs */
 
 typedef struct pod_attn_config {
   int32_t num_q_heads;      /* Hq */

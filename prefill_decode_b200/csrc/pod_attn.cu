@@ -66,6 +66,7 @@ struct alignas(64) PodParams {
   int32_t mode;
   int32_t use_tmem;
   int32_t merge_in_kernel; // 1: the warp finishing a row's last split merges the row
+  int32_t selftest_timeout; // 1: CTA 0 exercises the expired-wait path once
   float scale_log2;        // softmax scale * log2(e)
 };
 
@@ -111,7 +112,7 @@ struct Cfg {
   static constexpr int kSmem = kPrefillSmem;
   static constexpr int kNumBars = kBarDecode + kWarpsPerCta * kNS;
   static constexpr int kCtrlBytes = 512;                      // barriers, TMEM address, broadcast slots
-  static_assert(kNumBars * 8 + 32 <= kCtrlBytes, "control block too small");
+  static_assert((kNumBars + 1) * 8 + 32 <= kCtrlBytes, "control block too small");   // + the self-test barrier
   // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) can share an SM
   static constexpr int kSmemAlloc = (kSmem + kCtrlBytes) > 80 * 1024 ? (kSmem + kCtrlBytes) : 80 * 1024;
 };
@@ -693,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
   using CF = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + CF::kSmem);
-  uint32_t* ctrl = reinterpret_cast<uint32_t*>(bars + CF::kNumBars);   // TMEM address, home role, item, abort
+  uint32_t* ctrl = reinterpret_cast<uint32_t*>(bars + CF::kNumBars + 1);   // TMEM address, home role, item, abort
   volatile int* sh_abort = reinterpret_cast<volatile int*>(ctrl + 3);
   const int tid = threadIdx.x, warp = tid >> 5;
   if (smem_u32(smem) & 1023u) {   // the swizzled tiles need 1024-byte alignment
@@ -701,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
     return;
   }
   if (tid == 0) {
-    for (int i = 0; i < CF::kNumBars; ++i) {
+    for (int i = 0; i <= CF::kNumBars; ++i) {   // [kNumBars]: self-test barrier, never arrived at
       uint32_t count = 1;
       if (i == kBarPFull || i == kBarPFull + 1) count = kWarpsPerCta;
       mbar_init(&bars[i], count);
@@ -732,6 +733,10 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tmem = p.use_tmem ? ctrl[0] : 0u;
   const int home = (int)ctrl[1];
+  if (p.selftest_timeout && blockIdx.x == 0 && tid == 0) {
+    // nothing ever arrives at this barrier: the bounded wait must expire and report
+    if (!mbar_wait(&bars[CF::kNumBars], 0u, 1000000ull)) record_error(p, POD_ERR_TIMEOUT, -1);
+  }
 
   uint32_t tiles_done = 0, items_done = 0, seq = 0;
   uint8_t* ring = smem + (warp < kWarpsPerCta ? warp : 0) * CF::kNS * CF::kDecStage;
@@ -1037,6 +1042,7 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   prm.merge_items = reinterpret_cast<const int4*>(w + pl->off_merge);
   prm.merge_cnt = reinterpret_cast<int32_t*>(w + pl->off_merge_cnt);
   prm.merge_in_kernel = (pl->cfg.flags & POD_FLAG_MERGE_KERNEL) ? 0 : 1;
+  prm.selftest_timeout = (pl->cfg.flags & POD_FLAG_SELFTEST_TIMEOUT) ? 1 : 0;
   prm.part_o = reinterpret_cast<float*>(w + pl->off_part_o);
   prm.part_lse = reinterpret_cast<float*>(w + pl->off_part_lse);
   prm.trace = (pl->cfg.flags & POD_FLAG_TRACE) ? trace : nullptr;

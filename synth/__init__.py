@@ -139,10 +139,18 @@ class Batch:
         return self.k_pool.shape[0]
 
 
-def make_batch(w: Workload) -> Batch:
-    Hq, Hkv, d = w.num_q_heads, w.num_kv_heads, w.head_dim
-    P, C, B = w.prefill_len, w.prefill_ctx, w.num_decode
-    rng = np.random.default_rng(w.seed)
+@dataclasses.dataclass
+class Layout:
+    """Lengths and paged-block layout of a batch (draws 1 and 2 of the recipe)."""
+    kv_lens: np.ndarray       # int32 [1 + B]
+    block_table: np.ndarray   # int32 [1 + B, max_pages]
+    num_blocks: int
+    unused_blocks: np.ndarray # blocks no request references (poison)
+
+
+def make_layout(w: Workload, rng: Optional[np.random.Generator] = None) -> Layout:
+    B, P, C = w.num_decode, w.prefill_len, w.prefill_ctx
+    rng = np.random.default_rng(w.seed) if rng is None else rng
     dec = _draw_lengths(rng, w)
     kv_lens = np.concatenate([np.asarray([C + P if P > 0 else 0], dtype=np.int32), dec]).astype(np.int32)
     pages = (kv_lens.astype(np.int64) + PAGE - 1) // PAGE
@@ -157,6 +165,18 @@ def make_batch(w: Workload) -> Batch:
         n = int(pages[r])
         bt[r, :n] = perm[off:off + n]
         off += n
+    return Layout(kv_lens, bt, num_blocks, perm[used:])
+
+
+def make_batch(w: Workload) -> Batch:
+    Hq, Hkv, d = w.num_q_heads, w.num_kv_heads, w.head_dim
+    P, C, B = w.prefill_len, w.prefill_ctx, w.num_decode
+    rng = np.random.default_rng(w.seed)
+    lay = make_layout(w, rng)
+    kv_lens, bt, num_blocks = lay.kv_lens, lay.block_table, lay.num_blocks
+    pages = (kv_lens.astype(np.int64) + PAGE - 1) // PAGE
+    used = int(pages.sum())
+    perm_unused = lay.unused_blocks
     q_pre = _normal_bf16(rng, (P, Hq, d))
     q_dec = _normal_bf16(rng, (B, Hq, d))
     k_pool = _normal_bf16(rng, (num_blocks, Hkv, PAGE, d))
@@ -169,7 +189,7 @@ def make_batch(w: Workload) -> Batch:
             blk = bt[r, n - 1]
             k_pool[blk, :, L % PAGE:, :] = pk
             v_pool[blk, :, L % PAGE:, :] = pv
-    for blk in perm[used:]:
+    for blk in perm_unused:
         k_pool[blk] = pk
         v_pool[blk] = pv
     return Batch(w, q_pre, q_dec, k_pool, v_pool, bt, kv_lens, w.softmax_scale)

@@ -10,7 +10,60 @@ def bits_to_bf16(torch, a: np.ndarray, device="cuda"):
     return t.view(torch.bfloat16).to(device)
 
 
+class _LayoutBatch:
+    """Host-side description of a batch whose values live only on the GPU."""
+
+    def __init__(self, w, lay):
+        self.workload = w
+        self.kv_lens = lay.kv_lens
+        self.block_table = lay.block_table
+        self.num_blocks = lay.num_blocks
+        self.scale = w.softmax_scale
+        self.prefill_len = w.prefill_len
+        self.prefill_ctx = w.prefill_ctx
+
+    @property
+    def decode_lens(self):
+        return self.kv_lens[1:]
+
+
 class DeviceBatch:
+    @classmethod
+    def generated_on_device(cls, torch, w, device="cuda"):
+        """Same lengths, block layout and poison as synth.make_batch, but the
+        normal values are drawn on the GPU by torch.Generator(seed) (for large
+        performance-only batches; the values differ from the NumPy recipe)."""
+        import synth
+        lay = synth.make_layout(w)
+        gen = torch.Generator(device=device)
+        gen.manual_seed(w.seed)
+        Hq, Hkv, d, P, B = w.num_q_heads, w.num_kv_heads, w.head_dim, w.prefill_len, w.num_decode
+
+        def normal(*shape):
+            return torch.randn(*shape, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+        self = cls.__new__(cls)
+        self.b = _LayoutBatch(w, lay)
+        self.torch = torch
+        self.q_pre = normal(P, Hq, d) if P else None
+        self.q_dec = normal(B, Hq, d) if B else None
+        self.k = normal(lay.num_blocks, Hkv, synth.PAGE, d)
+        self.v = normal(lay.num_blocks, Hkv, synth.PAGE, d)
+        for r, L in enumerate(lay.kv_lens.tolist()):
+            n = (L + synth.PAGE - 1) // synth.PAGE
+            if n and L % synth.PAGE:
+                blk = int(lay.block_table[r, n - 1])
+                self.k[blk, :, L % synth.PAGE:, :] = synth.POISON_K
+                self.v[blk, :, L % synth.PAGE:, :] = synth.POISON_V
+        for blk in lay.unused_blocks.tolist():
+            self.k[blk] = synth.POISON_K
+            self.v[blk] = synth.POISON_V
+        self.bt = torch.from_numpy(lay.block_table).to(device)
+        self.lens = torch.from_numpy(lay.kv_lens).to(device)
+        self.o_pre = torch.empty_like(self.q_pre) if self.q_pre is not None else None
+        self.o_dec = torch.empty_like(self.q_dec) if self.q_dec is not None else None
+        return self
+
     def __init__(self, torch, b, device="cuda"):
         self.b = b
         w = b.workload
