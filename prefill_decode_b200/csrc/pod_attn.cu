@@ -321,17 +321,13 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
     tmem_ld32(tmem + t_lane + (t & 1u) * kBN + 32, s + 32);
     tmem_wait_ld();
     float mx = -INFINITY;        // row max of the raw scores; m below is in scaled (log2) units
-    if (j < full_tiles) {
-#pragma unroll
-      for (int k = 0; k < kBN; ++k) mx = fmaxf(mx, s[k]);
-    } else {
+    if (j >= full_tiles) {
       const int lim = row_limit - j * kBN;
 #pragma unroll
-      for (int k = 0; k < kBN; ++k) {
-        s[k] = k < lim ? s[k] : -INFINITY;
-        mx = fmaxf(mx, s[k]);
-      }
+      for (int k = 0; k < kBN; ++k) s[k] = k < lim ? s[k] : -INFINITY;
     }
+#pragma unroll
+    for (int k = 0; k < kBN / 2; ++k) mx = fmax3(mx, s[2 * k], s[2 * k + 1]);
     mx *= sl2;
     if (j == 0) {
       m = mx;
@@ -359,17 +355,21 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
         m = m_new;
       }
     }
-    float rs = 0.f;
-    const float neg_m = -m;
+    // exponent arguments and row sums two at a time (packed fp32 pairs)
+    const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m, -m);
+    uint64_t rs2 = f2_pack(0.f, 0.f);
     uint32_t pk[kBN / 2];
 #pragma unroll
     for (int k = 0; k < kBN / 2; ++k) {
-      const float e0 = ex2(fmaf(s[2 * k], sl2, neg_m));
-      const float e1 = ex2(fmaf(s[2 * k + 1], sl2, neg_m));
-      rs += e0 + e1;
+      float a0, a1;
+      f2_unpack(f2_fma(f2_pack(s[2 * k], s[2 * k + 1]), scale2, negm2), a0, a1);
+      const float e0 = ex2(a0), e1 = ex2(a1);
+      rs2 = f2_add(rs2, f2_pack(e0, e1));
       pk[k] = pack_bf16(e0, e1);
     }
-    l += rs;
+    float r0, r1;
+    f2_unpack(rs2, r0, r1);
+    l += r0 + r1;
     // P_t (bf16 pairs) over the first 32 columns of S_t: the A operand of P.V_t
     tmem_st32_u(tmem + t_lane + (t & 1u) * kBN, pk);
     tmem_wait_st();
