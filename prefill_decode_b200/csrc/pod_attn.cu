@@ -410,15 +410,17 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
 // rows so only the head dimension is padded), online softmax per head across
 // lanes, P^T moved into the B-operand layout with movmatrix, then
 // O^T[d x 8] += V_page^T . P^T.  Pages arrive by TMA into a kNS-deep ring.
+// The block ids of an item's pages are read 32 at a time, one per lane, a
+// window ahead of use, so refilling a ring slot never waits on a global load.
 template <int D>
 __device__ __forceinline__ void decode_issue_page(const PodParams& p, uint8_t* ring, uint64_t* wbars, uint32_t seq,
-                                                  int bt_row, int gpage, int kvh) {
+                                                  int blk, int kvh) {
   using CF = Cfg<D>;
   const int s = seq % CF::kNS;
   uint8_t* kbuf = ring + s * CF::kDecStage;
   uint64_t* bar = &wbars[s];
   mbar_arrive_expect_tx(bar, CF::kDecStage);
-  const int row = kv_row(p, __ldg(&p.block_table[(size_t)bt_row * p.bt_stride + gpage]), kvh);
+  const int row = kv_row(p, blk, kvh);
 #pragma unroll
   for (int h = 0; h < CF::kHalves; ++h) {
     tma_load_2d(kbuf + h * (kPage * 128), &p.tm_k, bar, h * 64, row);
@@ -433,63 +435,102 @@ __device__ __forceinline__ uint32_t swz(int row, int col_elem) {
 
 // One warp merges the split partials of merge item `midx` into bf16 outputs:
 // O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s (log2 domain).
-// Lane l owns d elements [4l, 4l + 4) (and +128 ... for larger d) of every head,
-// so each split costs one independent 16-byte load per head and lane.  The
-// partials were written by other warps of this launch: read them through L2.
-template <int D>
-__device__ void merge_row_warp(const PodParams& p, int midx) {
+// Lane l owns d elements [4l, 4l + 4) (and +128 ... for larger d) of every head.
+// The per-head maxima come from one lane-parallel pass over the S*G
+// log-sum-exps (contiguous, [S][G]); the weighted sum then loads U splits of
+// all G heads per round trip (16 independent 16-byte loads per lane), so a
+// row costs about 1 + S/U memory latencies.  The partials were written by
+// other warps of this launch: read them through L2.
+template <int D, int G>
+__device__ void merge_row_g(const PodParams& p, int r, int kvh, int first, int S) {
   constexpr int kV = D / 128 > 0 ? D / 128 : 1;   // float4 chunks per lane and head
+  constexpr int U = 16 / G > 0 ? 16 / G : 1;       // splits per round trip
   const int lane = threadIdx.x & 31;
-  const int4 mi = __ldg(&p.merge_items[midx]);
-  const int r = mi.x, kvh = mi.y, first = mi.z, S = mi.w;
-  const int g = p.g;
   const bool active = (lane * 4) < D;
-  float M[8], den[8];
-  float4 acc[8][kV];
+  const float* lse = p.part_lse + (size_t)first * G;
+  const int n = S * G;
+  float M[G];
 #pragma unroll
-  for (int h = 0; h < 8; ++h) {
-    M[h] = -INFINITY;
+  for (int h = 0; h < G; ++h) M[h] = -INFINITY;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const float v = i < n ? __ldcg(lse + i) : -INFINITY;
+    const int hi = i % G;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float x = hi == h ? v : -INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+      M[h] = fmaxf(M[h], x);
+    }
+  }
+  float den[G];
+  float4 acc[G][kV];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
     den[h] = 0.f;
 #pragma unroll
     for (int v = 0; v < kV; ++v) acc[h][v] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int s = 0; s < S; ++s)
+  for (int s0 = 0; s0 < S; s0 += U) {
+    float4 x[U][G][kV];
+    float l[U][G];
 #pragma unroll
-    for (int h = 0; h < 8; ++h)
-      if (h < g) M[h] = fmaxf(M[h], __ldcg(&p.part_lse[(size_t)(first + s) * g + h]));
-  for (int s = 0; s < S; ++s) {
+    for (int u = 0; u < U; ++u) {
+      const bool in = s0 + u < S;
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      if (h < g) {
-        const float w = ex2(__ldcg(&p.part_lse[(size_t)(first + s) * g + h]) - M[h]);
+      for (int h = 0; h < G; ++h) {
+        const size_t e = (size_t)(first + s0 + u) * G + h;
+        l[u][h] = in ? __ldcg(p.part_lse + e) : -INFINITY;
+        const float4* po = reinterpret_cast<const float4*>(p.part_o + e * D);
+#pragma unroll
+        for (int v = 0; v < kV; ++v)
+          x[u][h][v] = (in && active) ? __ldcg(&po[lane + 32 * v]) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float w = s0 + u < S ? ex2(l[u][h] - M[h]) : 0.f;
         den[h] += w;
-        const float4* po = reinterpret_cast<const float4*>(p.part_o + ((size_t)(first + s) * g + h) * D);
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
-          if (active) {
-            const float4 x = __ldcg(&po[lane + 32 * v]);
-            acc[h][v].x += w * x.x;
-            acc[h][v].y += w * x.y;
-            acc[h][v].z += w * x.z;
-            acc[h][v].w += w * x.w;
-          }
+          acc[h][v].x += w * x[u][h][v].x;
+          acc[h][v].y += w * x[u][h][v].y;
+          acc[h][v].z += w * x[u][h][v].z;
+          acc[h][v].w += w * x[u][h][v].w;
         }
       }
     }
   }
+  if (!active) return;
 #pragma unroll
-  for (int h = 0; h < 8; ++h) {
-    if (h < g && active) {
-      const float inv = 1.f / den[h];
-      __nv_bfloat16* ob = p.o_dec + ((size_t)r * p.Hq + kvh * g + h) * D;
+  for (int h = 0; h < G; ++h) {
+    const float inv = 1.f / den[h];
+    __nv_bfloat16* ob = p.o_dec + ((size_t)r * p.Hq + kvh * G + h) * D;
 #pragma unroll
-      for (int v = 0; v < kV; ++v) {
-        uint2 o;
-        o.x = pack_bf16(acc[h][v].x * inv, acc[h][v].y * inv);
-        o.y = pack_bf16(acc[h][v].z * inv, acc[h][v].w * inv);
-        *reinterpret_cast<uint2*>(ob + 4 * (lane + 32 * v)) = o;
-      }
+    for (int v = 0; v < kV; ++v) {
+      uint2 o;
+      o.x = pack_bf16(acc[h][v].x * inv, acc[h][v].y * inv);
+      o.y = pack_bf16(acc[h][v].z * inv, acc[h][v].w * inv);
+      *reinterpret_cast<uint2*>(ob + 4 * (lane + 32 * v)) = o;
     }
+  }
+}
+
+template <int D>
+__device__ void merge_row_warp(const PodParams& p, int midx) {
+  const int4 mi = __ldg(&p.merge_items[midx]);
+  switch (p.g) {
+    case 1: merge_row_g<D, 1>(p, mi.x, mi.y, mi.z, mi.w); break;
+    case 2: merge_row_g<D, 2>(p, mi.x, mi.y, mi.z, mi.w); break;
+    case 3: merge_row_g<D, 3>(p, mi.x, mi.y, mi.z, mi.w); break;
+    case 4: merge_row_g<D, 4>(p, mi.x, mi.y, mi.z, mi.w); break;
+    case 5: merge_row_g<D, 5>(p, mi.x, mi.y, mi.z, mi.w); break;
+    case 6: merge_row_g<D, 6>(p, mi.x, mi.y, mi.z, mi.w); break;
+    case 7: merge_row_g<D, 7>(p, mi.x, mi.y, mi.z, mi.w); break;
+    default: merge_row_g<D, 8>(p, mi.x, mi.y, mi.z, mi.w); break;
   }
 }
 
@@ -519,8 +560,18 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         e[2] = home_role;
         atomicAdd(&e[3], 1);
       }
+    }
+    // block ids: bt_cur holds pages [32 win, 32 win + 32) of the item, bt_nxt the next window
+    const int* bt_item = p.block_table + (size_t)(1 + r) * p.bt_stride + p0;
+    int bt_cur = lane < np ? __ldg(bt_item + lane) : 0;
+    int bt_nxt = 32 + lane < np ? __ldg(bt_item + 32 + lane) : 0;
+    int win = 0;
+    {
       const int pre = np < CF::kNS ? np : CF::kNS;
-      for (int j = 0; j < pre; ++j) decode_issue_page<D>(p, ring, wbars, seq + j, 1 + r, p0 + j, kvh);
+      for (int j = 0; j < pre; ++j) {
+        const int blk = __shfl_sync(0xffffffffu, bt_cur, j);
+        if (lane == 0) decode_issue_page<D>(p, ring, wbars, seq + j, blk, kvh);
+      }
     }
     // Q^T as the B operand: thread holds head n = lane/4, d pairs (lane%4)*2 (+8)
     uint32_t qf[D / 16][2];
@@ -611,8 +662,18 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         acc[mt][3] *= alB;
         mma_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
       }
-      __syncwarp();
-      if (lane == 0 && j + CF::kNS < np) decode_issue_page<D>(p, ring, wbars, sq + CF::kNS, 1 + r, p0 + j + CF::kNS, kvh);
+      const int jn = j + CF::kNS;
+      if (jn < np) {
+        if ((jn >> 5) > win) {     // next window; fetch the one after it
+          ++win;
+          bt_cur = bt_nxt;
+          const int pg = 32 * (win + 1) + lane;
+          bt_nxt = pg < np ? __ldg(bt_item + pg) : 0;
+        }
+        const int blk = __shfl_sync(0xffffffffu, bt_cur, jn & 31);
+        __syncwarp();
+        if (lane == 0) decode_issue_page<D>(p, ring, wbars, sq + CF::kNS, blk, kvh);
+      }
     }
     if (!ok) {
       // drain copies still in flight into this warp's ring before giving up

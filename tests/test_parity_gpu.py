@@ -67,6 +67,11 @@ SMALL = [
     synth.custom("decode_only", 8, 2, 128, 0, 0, [1, 16, 31, 4097, 9000], 9),
     synth.custom("prefill_only", 8, 2, 128, 257, 1500, [], 10),
     synth.custom("prefill_no_prior", 4, 1, 64, 200, 0, [40], 11),
+    # group sizes that do not divide a warp (the split merge is specialised per group size)
+    synth.custom("g3", 6, 2, 128, 150, 300, [700, 3000, 33], 13),
+    synth.custom("g5_d64", 10, 2, 64, 70, 90, [2600, 17], 14),
+    synth.custom("g6", 12, 2, 128, 64, 500, [4100, 260], 15),
+    synth.custom("g7", 28, 4, 128, 96, 200, [3500, 1, 640], 16),
 ]
 
 
