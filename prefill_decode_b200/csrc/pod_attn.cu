@@ -44,6 +44,8 @@ struct alignas(64) PodParams {
   CUtensorMap tm_k;    // K cache viewed as 2D [num_blocks*Hkv*16 rows, d], box {64, 16}, 128B swizzle
   CUtensorMap tm_v;    // V cache, same view
   CUtensorMap tm_q;    // Q prefill viewed as 3D [P][Hq][d], box {64, 1, 128}, 128B swizzle
+  CUtensorMap tm_kp;   // K cache as 3D [d/64 halves][rows][64]: one box {64, 16, d/64} = one whole page
+  CUtensorMap tm_vp;   // V cache, same view
   const __nv_bfloat16* q_dec;
   __nv_bfloat16* o_pre;
   __nv_bfloat16* o_dec;
@@ -80,12 +82,12 @@ enum : int {
   kBarKFull = 1,    // [3] K tile landed (TMA)                                  count 1 + tx
   kBarKEmpty = 4,   // [3] K slot free again: its S MMA finished (commit)       count 1
   kBarVFull = 7,    // [2] V tile landed (TMA)                                  count 1 + tx
-  kBarVEmpty = 9,   // [2] V slot free again: its P.V MMA finished (commit)     count 1
-  kBarSFull = 11,   // [2] S tile ready in TMEM buffer t&1 (commit)             count 1
-  kBarPFull = 13,   // [2] P tile stored over S in TMEM (and O rescaled)        count 4 (softmax warps)
-  kBarODone = 15,   // [2] P.V MMA of tile t finished, slot t&1 (commit)        count 1
-  kBarOFinal = 17,  // last P.V MMA of an item finished (commit)                count 1
-  kBarDecode = 18,  // [kWarpsPerCta * kNS] decode page rings                   count 1 + tx
+  kBarSFull = 9,    // [2] S tile ready in TMEM buffer t&1 (commit)             count 1
+  kBarPFull = 11,   // [2] P tile stored over S in TMEM (and O rescaled)        count 4 (softmax warps)
+  kBarODone = 13,   // [2] P.V MMA of tile t finished: TMEM buffer t&1 and      count 1
+                    //     V slot t&1 are free again (commit)
+  kBarOFinal = 15,  // last P.V MMA of an item finished (commit)                count 1
+  kBarDecode = 16,  // [kWarpsPerCta * kNS] decode page rings                   count 1 + tx
 };
 // Parity waits are only sound when the waiter knows the barrier is at most one
 // phase away from the one it waits for.  For key tile t (counted over the
@@ -93,8 +95,10 @@ enum : int {
 // (which read P_{t-2} from that buffer) finished, and P.V_t needs P_t, so
 // s_full, p_full and o_done can never run two phases ahead of their waiters;
 // the softmax waits for P.V of tile t-1 on o_done[(t-1)&1], whose previous
-// phase (tile t-3) finished before S_t was issued; the epilogue waits on
-// o_final, which completes once per item.
+// phase (tile t-3) finished before S_t was issued; the TMA warp waits on
+// o_done[t&1] before loading V_{t+2} into slot t&1, and P.V_{t+2} cannot
+// finish before that load; the epilogue waits on o_final, which completes
+// once per item.
 
 template <int D>
 struct Cfg {
@@ -204,7 +208,7 @@ __device__ bool prefill_tma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
       if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKEmpty + t % 3], (t / 3) & 1u, kWaitLimitNs))) return false;
       issue_tile<D>(&p.tm_k, sm.k(t + CF::kKSlots), &bars[kBarKFull + t % 3], rk, lane);
     }
-    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarVEmpty + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs))) return false;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs))) return false;
     issue_tile<D>(&p.tm_v, sm.v(t + CF::kVSlots), &bars[kBarVFull + (t & 1u)], rv, lane);
   }
   return true;
@@ -276,7 +280,6 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
         umma_bf16_tmem_a(tmem + kTmemO, pa + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_o,
                          (j > 0 || kk > 0) ? 1u : 0u);
       umma_commit(&bars[kBarODone + (t & 1u)]);
-      umma_commit(&bars[kBarVEmpty + (t & 1u)]);
       if (j == nkb - 1) umma_commit(&bars[kBarOFinal]);
     }
     __syncwarp();
@@ -421,11 +424,10 @@ __device__ __forceinline__ void decode_issue_page(const PodParams& p, uint8_t* r
   uint64_t* bar = &wbars[s];
   mbar_arrive_expect_tx(bar, CF::kDecStage);
   const int row = kv_row(p, blk, kvh);
-#pragma unroll
-  for (int h = 0; h < CF::kHalves; ++h) {
-    tma_load_2d(kbuf + h * (kPage * 128), &p.tm_k, bar, h * 64, row);
-    tma_load_2d(kbuf + CF::kPageBytes + h * (kPage * 128), &p.tm_v, bar, h * 64, row);
-  }
+  // one box per page of K and of V: both 64-element halves of 16 rows land as
+  // [half][16 rows][128 B], the layout two 2D boxes would give
+  tma_load_3d(kbuf, &p.tm_kp, bar, 0, row, 0);
+  tma_load_3d(kbuf + CF::kPageBytes, &p.tm_vp, bar, 0, row, 0);
 }
 
 __device__ __forceinline__ uint32_t swz(int row, int col_elem) {
@@ -772,6 +774,8 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
     *sh_abort = 0;
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
+    tma_prefetch_desc(&p.tm_kp);
+    tma_prefetch_desc(&p.tm_vp);
     int home = p.mode == kDecodeOnly ? kRoleDecode : kRolePrefill;
     if (p.mode == kFused) {
       const uint32_t sm = smid();
@@ -1080,6 +1084,18 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
                       es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r1 != CUDA_SUCCESS || r2 != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
+    // page view: x = element within a 64-element half, y = row, z = half (row stride 2d bytes, half stride 128 B)
+    const cuuint64_t pdims[3] = {64, (cuuint64_t)num_blocks * Hkv * kPage, (cuuint64_t)(D / 64)};
+    const cuuint64_t pstrides[2] = {(cuuint64_t)D * 2, 128};
+    const cuuint32_t pbox[3] = {64, (cuuint32_t)kPage, (cuuint32_t)(D / 64)};
+    const cuuint32_t pes[3] = {1, 1, 1};
+    CUresult r3 = enc(&prm.tm_kp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache), pdims, pstrides, pbox,
+                      pes, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r4 = enc(&prm.tm_vp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(v_cache), pdims, pstrides, pbox,
+                      pes, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r3 != CUDA_SUCCESS || r4 != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
   }
   if (has_pre) {
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)pl->P};
