@@ -16,8 +16,9 @@
 // B200 re-design (prior art, not the blueprint): CTAs are persistent -- the
 // ticket fixes a CTA's home role, the CTA drains that role's queue and then
 // steals from the other, so no CTA ever waits on another.  Prefill tiles are
-// 128 x 64 tcgen05 MMAs with S and P.V accumulated in TMEM, fed by TMA with
-// 128-byte swizzle straight from the 16-token pages; decode warps stage pages
+// 128 x 64 tcgen05 MMAs: S = Q K^T with Q held in TMEM, O += P V with P staged
+// in shared memory, both accumulated in TMEM; K and V arrive by TMA with
+// 128-byte swizzle straight from the 16-token pages.  Decode warps stage pages
 // with TMA into a per-warp ring and use m16n8k16 MMAs with keys as rows.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -34,7 +35,9 @@
 namespace pod {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a healthy wait takes microseconds
-constexpr uint32_t kTmemCols = 256;                // S double buffer (2 x 64 cols) at 0, O (d cols) at 128
+constexpr uint32_t kTmemCols = 256;   // S (64 fp32 columns) at 0, Q (d/2 columns of bf16 pairs) at 64, O (d) at 128
+constexpr uint32_t kTmemS = 0;
+constexpr uint32_t kTmemQ = 64;
 constexpr uint32_t kTmemO = 128;
 
 enum Mode : int32_t { kFused = 0, kPrefillOnly = 1, kDecodeOnly = 2 };
@@ -42,10 +45,9 @@ enum Role : int32_t { kRolePrefill = 0, kRoleDecode = 1 };
 
 struct alignas(64) PodParams {
   CUtensorMap tm_k;    // K cache viewed as 2D [num_blocks*Hkv*16 rows, d], box {64, 16}, 128B swizzle
-  CUtensorMap tm_v;    // V cache, same view
-  CUtensorMap tm_q;    // Q prefill viewed as 3D [P][Hq][d], box {64, 1, 128}, 128B swizzle
   CUtensorMap tm_kp;   // K cache as 3D [d/64 halves][rows][64]: one box {64, 16, d/64} = one whole page
   CUtensorMap tm_vp;   // V cache, same view
+  const __nv_bfloat16* q_pre;
   const __nv_bfloat16* q_dec;
   __nv_bfloat16* o_pre;
   __nv_bfloat16* o_dec;
@@ -78,38 +80,40 @@ constexpr int kTmaWarp = 5;
 
 // mbarrier slots in the CTA control block
 enum : int {
-  kBarQ = 0,        // Q tile landed (TMA)                                      count 1 + tx
+  kBarQ = 0,        // Q rows of the item stored into TMEM                      count 4 (softmax warps)
   kBarKFull = 1,    // [3] K tile landed (TMA)                                  count 1 + tx
   kBarKEmpty = 4,   // [3] K slot free again: its S MMA finished (commit)       count 1
   kBarVFull = 7,    // [2] V tile landed (TMA)                                  count 1 + tx
-  kBarSFull = 9,    // [2] S tile ready in TMEM buffer t&1 (commit)             count 1
-  kBarPFull = 11,   // [2] P tile stored over S in TMEM (and O rescaled)        count 4 (softmax warps)
-  kBarODone = 13,   // [2] P.V MMA of tile t finished: TMEM buffer t&1 and      count 1
-                    //     V slot t&1 are free again (commit)
+  kBarSFull = 9,    // S tile ready in TMEM (commit)                            count 1
+  kBarSFree = 10,   // softmax has read S out of TMEM                           count 4 (softmax warps)
+  kBarPFull = 11,   // [2] P tile t stored in shared-memory buffer t&1          count 4 (softmax warps)
+  kBarODone = 13,   // [2] P.V MMA of tile t finished: P buffer and V slot t&1  count 1
+                    //     are free again (commit)
   kBarOFinal = 15,  // last P.V MMA of an item finished (commit)                count 1
   kBarDecode = 16,  // [kWarpsPerCta * kNS] decode page rings                   count 1 + tx
 };
 // Parity waits are only sound when the waiter knows the barrier is at most one
 // phase away from the one it waits for.  For key tile t (counted over the
-// CTA's lifetime): S_t goes into TMEM buffer t&1 only after P.V of tile t-2
-// (which read P_{t-2} from that buffer) finished, and P.V_t needs P_t, so
-// s_full, p_full and o_done can never run two phases ahead of their waiters;
-// the softmax waits for P.V of tile t-1 on o_done[(t-1)&1], whose previous
-// phase (tile t-3) finished before S_t was issued; the TMA warp waits on
-// o_done[t&1] before loading V_{t+2} into slot t&1, and P.V_{t+2} cannot
-// finish before that load; the epilogue waits on o_final, which completes
-// once per item.
+// CTA's lifetime): S_{t+1} is issued only after the softmax has read S_t
+// (s_free), and the softmax reads S_{t+1} only after S_t, so s_full and s_free
+// alternate; K_{t+3} is loaded into slot t%3 after S_t finished (k_empty) and
+// S_{t+3} needs it; P_t goes into buffer t&1 only after P.V_{t-2} finished and
+// P.V_t needs P_t, so p_full is at most one phase ahead per buffer; o_done[t&1]
+// is waited on by the TMA warp (before V_{t+2} goes into slot t&1) and by the
+// softmax (tiles t+1 and t+2, before it rescales O or reuses the P buffer),
+// and P.V_{t+2} needs both; q and o_final complete once per item.
 
 template <int D>
 struct Cfg {
   static constexpr int kHalves = D / 64;                      // 128-byte swizzle atoms along d
-  static constexpr int kQBytes = kBM * D * 2;                 // 128 query rows
   static constexpr int kKTile = kBN * D * 2;                  // 64 keys of K (or V)
   static constexpr int kKSlots = 3;                           // K ring: two tiles of lead
   static constexpr int kVSlots = 2;                           // V ring: two tiles of lead
-  static constexpr int kOffK = kQBytes;
+  static constexpr int kPBytes = kBM * kBN * 2;               // P tile, bf16, K-major 128B-swizzled
+  static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kKSlots * kKTile;
-  static constexpr int kPrefillSmem = kOffV + kVSlots * kKTile;
+  static constexpr int kOffP = kOffV + kVSlots * kKTile;      // [2] P buffers
+  static constexpr int kPrefillSmem = kOffP + 2 * kPBytes;
   static constexpr int kPageBytes = kPage * D * 2;            // one 16-token page of one kv head
   static constexpr int kDecStage = 2 * kPageBytes;            // K page + V page
   static constexpr int kNS = (kPrefillSmem / kWarpsPerCta) / kDecStage;   // decode ring depth per warp
@@ -143,19 +147,31 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 template <int D>
 struct PrefillSmem {
   uint8_t* base;
-  __device__ uint8_t* q() const { return base; }
   __device__ uint8_t* k(uint32_t t) const { return base + Cfg<D>::kOffK + (t % Cfg<D>::kKSlots) * Cfg<D>::kKTile; }
   __device__ uint8_t* v(uint32_t t) const { return base + Cfg<D>::kOffV + (t % Cfg<D>::kVSlots) * Cfg<D>::kKTile; }
+  __device__ uint8_t* pbuf(uint32_t t) const { return base + Cfg<D>::kOffP + (t & 1u) * Cfg<D>::kPBytes; }
 };
 
-// TMA warp: tensor-map rows of the 4 pages of key tile kb (lanes 0..3 look the
-// block ids up in parallel; pages past kv_end read past the tensor's end =
-// zeros).  Returns the row of page `lane & 3` in every lane.
-__device__ __forceinline__ int tile_page_row(const PodParams& p, int kb, int kvh, int kv_end, int lane) {
+// Block ids of the prefill request's pages, read 32 at a time (one per lane) a
+// window ahead of use: `cur` holds pages [32 w, 32 w + 32) (key tiles 8w ..
+// 8w + 7), `nxt` the next 32.
+struct PageWindows {
+  int cur, nxt, w;
+};
+
+__device__ __forceinline__ int load_page_window(const PodParams& p, int w, int kv_end, int lane) {
+  const int gp = 32 * w + lane;
+  return gp * kPage < kv_end ? __ldg(&p.block_table[gp]) : 0;
+}
+
+// Tensor-map row of page `lane & 3` of key tile kb (kb in window w or w + 1);
+// pages past kv_end map past the tensor's end, where TMA reads zeros.
+__device__ __forceinline__ int tile_page_row(const PodParams& p, const PageWindows& pw, int kb, int kvh, int kv_end,
+                                             int lane) {
+  const int src = (kb >> 3) == pw.w ? pw.cur : pw.nxt;
+  const int blk = __shfl_sync(0xffffffffu, src, ((kb & 7) << 2) + (lane & 3));
   const int gp = kb * (kBN / kPage) + (lane & 3);
-  int row = p.kv_rows;
-  if (lane < 4 && gp * kPage < kv_end) row = kv_row(p, __ldg(&p.block_table[gp]), kvh);
-  return row;
+  return gp * kPage < kv_end ? kv_row(p, blk, kvh) : p.kv_rows;
 }
 
 template <int D>
@@ -175,49 +191,67 @@ __device__ __forceinline__ void issue_tile(const CUtensorMap* map, uint8_t* dst,
   }
 }
 
-// TMA warp of one prefill item: Q, then K into a 3-deep ring and V into a
-// 2-deep ring, refilling a slot as soon as the MMA warp reports its P.V done.
-// `t0` = key tiles this CTA processed before this item (it indexes every ring
-// and mbarrier phase).
+// V tile of 4 pages as one page box each ([page][d/64 halves][16 rows][128 B]);
+// a P.V MMA step of 16 keys reads exactly one page, so the page-major layout
+// only changes the B descriptor's strides.
+template <int D>
+__device__ __forceinline__ void issue_vtile(const PodParams& p, uint8_t* dst, uint64_t* bar, int row_lane, int lane) {
+  using CF = Cfg<D>;
+  int rows[kBN / kPage];
+#pragma unroll
+  for (int pi = 0; pi < kBN / kPage; ++pi) rows[pi] = __shfl_sync(0xffffffffu, row_lane, pi);
+  if (lane == 0) {
+    mbar_arrive_expect_tx(bar, CF::kKTile);
+#pragma unroll
+    for (int pi = 0; pi < kBN / kPage; ++pi) tma_load_3d(dst + pi * CF::kPageBytes, &p.tm_vp, bar, 0, rows[pi], 0);
+  }
+}
+
+// TMA warp of one prefill item: K into a 3-deep ring and V into a 2-deep
+// ring; K_{t+3} goes into slot t%3 once S_t finished, V_{t+2} into slot t&1
+// once P.V_t finished.  `t0` = key tiles this CTA processed before this item
+// (it indexes every ring and mbarrier phase).
 template <int D>
 __device__ bool prefill_tma(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t t0) {
   using CF = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  const int q0 = it.x, qh = it.y, kv_end = it.z;
+  const int qh = it.y, kv_end = it.z;
   const int kvh = qh / p.g;
   const int nkb = (kv_end + kBN - 1) / kBN;
   const PrefillSmem<D> sm{smem};
-  if (lane == 0) {
-    if (p.kv_lens && __ldg(&p.kv_lens[0]) < kv_end) record_error(p, POD_ERR_PLAN_MISMATCH, 0);
-    mbar_arrive_expect_tx(&bars[kBarQ], CF::kQBytes);
-#pragma unroll
-    for (int h = 0; h < CF::kHalves; ++h) tma_load_3d(sm.q() + h * (kBM * 128), &p.tm_q, &bars[kBarQ], h * 64, qh, q0);
-  }
+  if (lane == 0 && p.kv_lens && __ldg(&p.kv_lens[0]) < kv_end) record_error(p, POD_ERR_PLAN_MISMATCH, 0);
+  PageWindows pw{load_page_window(p, 0, kv_end, lane), load_page_window(p, 1, kv_end, lane), 0};
   for (int j = 0; j < nkb && j < CF::kKSlots; ++j) {
     const uint32_t t = t0 + j;
-    const int r = tile_page_row(p, j, kvh, kv_end, lane);
+    const int r = tile_page_row(p, pw, j, kvh, kv_end, lane);
     issue_tile<D>(&p.tm_k, sm.k(t), &bars[kBarKFull + t % 3], r, lane);
-    if (j < CF::kVSlots) issue_tile<D>(&p.tm_v, sm.v(t), &bars[kBarVFull + (t & 1u)], r, lane);
+    if (j < CF::kVSlots) issue_vtile<D>(p, sm.v(t), &bars[kBarVFull + (t & 1u)], r, lane);
   }
   for (int j = 0; j + CF::kVSlots < nkb; ++j) {
     const uint32_t t = t0 + j;
+    if (((j + CF::kVSlots) >> 3) > pw.w) {   // tile j+2 enters the next window; fetch the one after it
+      ++pw.w;
+      pw.cur = pw.nxt;
+      pw.nxt = load_page_window(p, pw.w + 1, kv_end, lane);
+    }
     const bool more_k = j + CF::kKSlots < nkb;
-    const int rk = more_k ? tile_page_row(p, j + CF::kKSlots, kvh, kv_end, lane) : 0;
-    const int rv = tile_page_row(p, j + CF::kVSlots, kvh, kv_end, lane);
-    if (more_k) {                // K first: the MMA warp needs it two tiles ahead
+    const int rk = more_k ? tile_page_row(p, pw, j + CF::kKSlots, kvh, kv_end, lane) : 0;
+    const int rv = tile_page_row(p, pw, j + CF::kVSlots, kvh, kv_end, lane);
+    if (more_k) {                // K first: S_{t+3} is issued well before P.V_{t+2}
       if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKEmpty + t % 3], (t / 3) & 1u, kWaitLimitNs))) return false;
       issue_tile<D>(&p.tm_k, sm.k(t + CF::kKSlots), &bars[kBarKFull + t % 3], rk, lane);
     }
     if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs))) return false;
-    issue_tile<D>(&p.tm_v, sm.v(t + CF::kVSlots), &bars[kBarVFull + (t & 1u)], rv, lane);
+    issue_vtile<D>(p, sm.v(t + CF::kVSlots), &bars[kBarVFull + (t & 1u)], rv, lane);
   }
   return true;
 }
 
-// MMA warp of one prefill item (lane 0 issues): S_t = Q K_t^T into TMEM buffer
-// t&1, two tiles ahead of the softmax; O += P_t V_t with P_t read from TMEM
-// (stored by the softmax over the first 32 columns of S_t).  Commits free the
-// K slot right after S_t and the V slot and the TMEM buffer after P.V_t.
+// MMA warp of one prefill item (lane 0 issues): S_t = Q K_t^T into TMEM with Q
+// read from TMEM (stored there by the softmax warps), issued as soon as the
+// softmax has read S_{t-1} out; O += P_t V_t with P_t read from shared memory.
+// Commits free the K slot right after S_t and the V slot and the P buffer
+// after P.V_t.
 template <int D>
 __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t tmem, uint32_t t0,
                             uint32_t nq) {
@@ -229,34 +263,45 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
   constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false, false);
   constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, false, true);
   // descriptors of the slot bases; a byte offset b within a slot adds b >> 4
-  const uint64_t dq = sdesc_sw128(smem_u32(sm.q()), 16, 1024);
   const uint64_t dk0 = sdesc_sw128(smem_u32(smem + CF::kOffK), 16, 1024);
-  const uint64_t dv0 = sdesc_sw128(smem_u32(smem + CF::kOffV), kBN * 128, 1024);
+  // V: MN-major, halves of d 16*128 bytes apart inside a page, 8-key groups 1024 apart
+  const uint64_t dv0 = sdesc_sw128(smem_u32(smem + CF::kOffV), kPage * 128, 1024);
+  const uint64_t dp0 = sdesc_sw128(smem_u32(smem + CF::kOffP), 16, 1024);
 
   auto issue_s = [&](uint32_t t) {
     const uint64_t dk = dk0 + (uint64_t)(((t % CF::kKSlots) * CF::kKTile) >> 4);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t aoff = ((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4;
       const uint32_t boff = ((kk >> 2) * (kBN * 128) + (kk & 3) * 32) >> 4;
-      umma_bf16(tmem + (t & 1u) * kBN, dq + aoff, dk + boff, idesc_s, kk > 0 ? 1u : 0u);
+      umma_bf16_tmem_a(tmem + kTmemS, tmem + kTmemQ + kk * 8, dk + boff, idesc_s, kk > 0 ? 1u : 0u);
     }
-    umma_commit(&bars[kBarSFull + (t & 1u)]);
+    umma_commit(&bars[kBarSFull]);
     umma_commit(&bars[kBarKEmpty + t % 3]);
   };
 
-  if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarQ], nq & 1u, kWaitLimitNs))) return false;
-  for (int i = 0; i < 2 && i < nkb; ++i) {   // S of the first two tiles
-    const uint32_t tn = t0 + i;
-    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKFull + tn % 3], (tn / 3) & 1u, kWaitLimitNs))) return false;
+  {                              // S of the first tile, once Q is in TMEM
+    const bool ok = mbar_wait(&bars[kBarQ], nq & 1u, kWaitLimitNs) &&
+                    mbar_wait(&bars[kBarKFull + t0 % 3], (t0 / 3) & 1u, kWaitLimitNs);
+    if (!__all_sync(0xffffffffu, ok)) return false;
     if (lane == 0) {
       tc_fence_after();
-      issue_s(tn);
+      issue_s(t0);
     }
     __syncwarp();
   }
   for (int j = 0; j < nkb; ++j) {
     const uint32_t t = t0 + j;
+    if (j + 1 < nkb) {           // S_{t+1} once the softmax has read S_t out of TMEM
+      const uint32_t tn = t + 1;
+      const bool ws = mbar_wait(&bars[kBarSFree], t & 1u, kWaitLimitNs) &&
+                      mbar_wait(&bars[kBarKFull + tn % 3], (tn / 3) & 1u, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ws)) return false;
+      if (lane == 0) {
+        tc_fence_after();
+        issue_s(tn);
+      }
+      __syncwarp();
+    }
     const bool wp = mbar_wait(&bars[kBarVFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs) &&
                     mbar_wait(&bars[kBarPFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs);
     if (!__all_sync(0xffffffffu, wp)) return false;
@@ -266,7 +311,8 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
       for (int i = lane; i < (kBN - valid) * CF::kHalves * 8; i += 32) {
         const int chunk = i & 7, rh = i >> 3;
         const int key = valid + rh % (kBN - valid), h = rh / (kBN - valid);
-        *reinterpret_cast<uint4*>(vt + h * (kBN * 128) + key * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(vt + (key / kPage) * CF::kPageBytes + h * (kPage * 128) + (key % kPage) * 128 +
+                                  chunk * 16) = make_uint4(0, 0, 0, 0);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -274,34 +320,25 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
     if (lane == 0) {
       tc_fence_after();
       const uint64_t dv = dv0 + (uint64_t)(((t & 1u) * CF::kKTile) >> 4);
-      const uint32_t pa = tmem + (t & 1u) * kBN;
+      const uint64_t dp = dp0 + (uint64_t)(((t & 1u) * CF::kPBytes) >> 4);
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk)
-        umma_bf16_tmem_a(tmem + kTmemO, pa + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_o,
-                         (j > 0 || kk > 0) ? 1u : 0u);
+        umma_bf16(tmem + kTmemO, dp + (uint64_t)((kk * 32) >> 4), dv + (uint64_t)((kk * CF::kPageBytes) >> 4), idesc_o,
+                  (j > 0 || kk > 0) ? 1u : 0u);
       umma_commit(&bars[kBarODone + (t & 1u)]);
       if (j == nkb - 1) umma_commit(&bars[kBarOFinal]);
     }
     __syncwarp();
-    if (j + 2 < nkb) {           // S_{t+2} into buffer t&1 once P.V_t has read P_t from it
-      const uint32_t tn = t + 2;
-      const bool ws = mbar_wait(&bars[kBarODone + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs) &&
-                      mbar_wait(&bars[kBarKFull + tn % 3], (tn / 3) & 1u, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, ws)) return false;
-      if (lane == 0) {
-        tc_fence_after();
-        issue_s(tn);
-      }
-      __syncwarp();
-    }
   }
   return true;
 }
 
 // Softmax warps of one prefill item (threads 0..127, thread = tile row = TMEM
-// lane).  Per key tile: read S_t from TMEM, mask (bottom-right causal), online
-// softmax in the exp2 domain with a lazily updated row max (O in TMEM is
-// rescaled only when the max grows by more than 2^8), write P_t as bf16 in the
+// lane).  First the thread's Q row goes into TMEM (the A operand of S = Q K^T).
+// Per key tile: read S_t from TMEM (and hand the buffer back to the MMA warp
+// at once), mask (bottom-right causal), online softmax in the exp2 domain with
+// a lazily updated row max (O in TMEM is rescaled only when the max grows by
+// more than 2^8), write P_t as bf16 into shared-memory buffer t&1 in the
 // K-major 128B-swizzled layout; finally O / l -> bf16 -> global.
 template <int D>
 __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t tmem,
@@ -314,15 +351,42 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
   const int full_tiles = (p.C + q0 + 1) / kBN;   // tiles visible to every row of this item
   const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
   const float sl2 = p.scale_log2;
+  {
+    // Q row (bf16 pairs along d) into TMEM lane `row`; rows past the chunk are zero
+    const int q = q0 + row;
+    const uint4* src = reinterpret_cast<const uint4*>(p.q_pre + ((size_t)q * p.Hq + qh) * D);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      uint32_t w[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = q < p.P ? __ldg(src + c * 8 + i) : make_uint4(0u, 0u, 0u, 0u);
+        w[4 * i] = v.x;
+        w[4 * i + 1] = v.y;
+        w[4 * i + 2] = v.z;
+        w[4 * i + 3] = v.w;
+      }
+      tmem_st32_u(tmem + t_lane + kTmemQ + c * 32, w);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[kBarQ]);
+  }
   float m = -INFINITY, l = 0.f;
   for (int j = 0; j < nkb; ++j) {
     const uint32_t t = t0 + j;
-    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs))) return false;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull], t & 1u, kWaitLimitNs))) return false;
     tc_fence_after();
     float s[kBN];
-    tmem_ld32(tmem + t_lane + (t & 1u) * kBN, s);
-    tmem_ld32(tmem + t_lane + (t & 1u) * kBN + 32, s + 32);
+    tmem_ld32(tmem + t_lane + kTmemS, s);
+    tmem_ld32(tmem + t_lane + kTmemS + 32, s + 32);
     tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[kBarSFree]);   // S_{t+1} may overwrite the buffer now
+    // P.V of tile t-2 read P buffer t&1; tiles of an earlier item finished with it
+    bool pbuf_free = j < 2;
     float mx = -INFINITY;        // row max of the raw scores; m below is in scaled (log2) units
     if (j >= full_tiles) {
       const int lim = row_limit - j * kBN;
@@ -341,6 +405,7 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
         const uint32_t tp = t - 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone + (tp & 1u)], (tp >> 1) & 1u, kWaitLimitNs)))
           return false;
+        pbuf_free = true;        // P.V MMAs finish in issue order
         tc_fence_after();
         const float m_new = need ? mx : m;
         const float alpha = ex2(m - m_new);
@@ -373,9 +438,18 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
     float r0, r1;
     f2_unpack(rs2, r0, r1);
     l += r0 + r1;
-    // P_t (bf16 pairs) over the first 32 columns of S_t: the A operand of P.V_t
-    tmem_st32_u(tmem + t_lane + (t & 1u) * kBN, pk);
-    tmem_wait_st();
+    // P_t into shared P buffer t&1 (the A operand of P.V_t) once P.V_{t-2} has read it
+    if (!pbuf_free) {
+      const uint32_t tp = t - 2;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone + (tp & 1u)], (tp >> 1) & 1u, kWaitLimitNs)))
+        return false;
+    }
+    uint8_t* prow = smem + Cfg<D>::kOffP + (t & 1u) * Cfg<D>::kPBytes + row * 128;   // 128 B, swizzled
+#pragma unroll
+    for (int c = 0; c < kBN / 8; ++c)
+      *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
+          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+    fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core's reads
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars[kBarPFull + (t & 1u)]);
@@ -767,13 +841,12 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
   if (tid == 0) {
     for (int i = 0; i <= CF::kNumBars; ++i) {   // [kNumBars]: self-test barrier, never arrived at
       uint32_t count = 1;
-      if (i == kBarPFull || i == kBarPFull + 1) count = kWarpsPerCta;
+      if (i == kBarQ || i == kBarSFree || i == kBarPFull || i == kBarPFull + 1) count = kWarpsPerCta;
       mbar_init(&bars[i], count);
     }
     fence_mbar_init();
     *sh_abort = 0;
     tma_prefetch_desc(&p.tm_k);
-    tma_prefetch_desc(&p.tm_v);
     tma_prefetch_desc(&p.tm_kp);
     tma_prefetch_desc(&p.tm_vp);
     int home = p.mode == kDecodeOnly ? kRoleDecode : kRolePrefill;
@@ -1080,10 +1153,7 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
     CUresult r1 = enc(&prm.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_cache), dims, strides, box,
                       es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    CUresult r2 = enc(&prm.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(v_cache), dims, strides, box,
-                      es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r1 != CUDA_SUCCESS || r2 != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
+    if (r1 != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
     // page view: x = element within a 64-element half, y = row, z = half (row stride 2d bytes, half stride 128 B)
     const cuuint64_t pdims[3] = {64, (cuuint64_t)num_blocks * Hkv * kPage, (cuuint64_t)(D / 64)};
     const cuuint64_t pstrides[2] = {(cuuint64_t)D * 2, 128};
@@ -1097,17 +1167,8 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r3 != CUDA_SUCCESS || r4 != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
   }
-  if (has_pre) {
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)pl->P};
-    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
-    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kBM};
-    const cuuint32_t es[3] = {1, 1, 1};
-    CUresult r = enc(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q_prefill), dims, strides, box,
-                     es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
-  }
   uint8_t* w = static_cast<uint8_t*>(ws);
+  prm.q_pre = static_cast<const __nv_bfloat16*>(q_prefill);
   prm.q_dec = static_cast<const __nv_bfloat16*>(q_decode);
   prm.o_pre = static_cast<__nv_bfloat16*>(o_prefill);
   prm.o_dec = static_cast<__nv_bfloat16*>(o_decode);
