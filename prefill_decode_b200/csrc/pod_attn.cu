@@ -627,26 +627,28 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
     const int r = a.x, kvh = a.y, k0 = a.z, k1 = a.w, part = b.x, midx = b.y, nsplit = b.z;
     const int p0 = k0 / kPage;
     const int np = (k1 - k0 + kPage - 1) / kPage;
-    if (lane == 0) {
-      if (p.kv_lens && __ldg(&p.kv_lens[1 + r]) < k1) record_error(p, POD_ERR_PLAN_MISMATCH, item);
-      if (p.trace) {
-        int32_t* e = p.trace + 4 * (p.n_pre + item);
-        e[0] = (int32_t)smid();
-        e[1] = blockIdx.x;
-        e[2] = home_role;
-        atomicAdd(&e[3], 1);
-      }
-    }
-    // block ids: bt_cur holds pages [32 win, 32 win + 32) of the item, bt_nxt the next window
+    // block ids: bt_cur holds pages [32 win, 32 win + 32) of the item, bt_nxt the next window;
+    // the request's length is read in the same round trip and checked once the pages are under way
     const int* bt_item = p.block_table + (size_t)(1 + r) * p.bt_stride + p0;
     int bt_cur = lane < np ? __ldg(bt_item + lane) : 0;
     int bt_nxt = 32 + lane < np ? __ldg(bt_item + 32 + lane) : 0;
+    const int len_now = (lane == 0 && p.kv_lens) ? __ldg(&p.kv_lens[1 + r]) : k1;
     int win = 0;
     {
       const int pre = np < CF::kNS ? np : CF::kNS;
       for (int j = 0; j < pre; ++j) {
         const int blk = __shfl_sync(0xffffffffu, bt_cur, j);
         if (lane == 0) decode_issue_page<D>(p, ring, wbars, seq + j, blk, kvh);
+      }
+    }
+    if (lane == 0) {
+      if (len_now < k1) record_error(p, POD_ERR_PLAN_MISMATCH, item);
+      if (p.trace) {
+        int32_t* e = p.trace + 4 * (p.n_pre + item);
+        e[0] = (int32_t)smid();
+        e[1] = blockIdx.x;
+        e[2] = home_role;
+        atomicAdd(&e[3], 1);
       }
     }
     // Q^T as the B operand: thread holds head n = lane/4, d pairs (lane%4)*2 (+8)
