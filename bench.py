@@ -44,11 +44,18 @@ KERNEL_SOURCES = ["prefill_decode_b200/csrc/pod_attn.cu", "prefill_decode_b200/c
                   "prefill_decode_b200/csrc/pod_plan.h"]
 
 
-def kernel_source_sha() -> str:
+HOST_SIDE_MARKER = b"// =========================================================== host side (ABI)"
+
+
+def kernel_source_sha(root: str = ROOT) -> str:
+    """Hash of the device code: the kernel sources, with the host-side ABI part
+    of the .cu file (launch plumbing, tensor-map encoding) left out."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(root, f), "rb") as fh:
+            data = fh.read()
+        i = data.find(HOST_SIDE_MARKER)
+        h.update(data if i < 0 else data[:i])
     return h.hexdigest()[:16]
 
 
@@ -241,7 +248,7 @@ def config_dict(w, b, mode):
 
 # ---------------------------------------------------------------- sweep mode
 def run_sweep(args):
-    """Every named workload and every mix-sweep point (fused and sequential),
+    """Every named workload and every mix-sweep point (fused, sequential, two streams),
     one JSON object per line; for the committed result tables, not the bench
     line the contract reads."""
     import torch
@@ -258,7 +265,8 @@ def run_sweep(args):
     for w in wls:
         db = DeviceBatch.generated_on_device(torch, w)
         res = {"workload": w.name, "values": "torch.Generator(cuda, seed) normals; layout from synth"}
-        for mode, flags in (("fused", 0), ("sequential", pod.POD_FLAG_SEQUENTIAL)):
+        for mode, flags in (("fused", 0), ("sequential", pod.POD_FLAG_SEQUENTIAL),
+                            ("two_streams", pod.POD_FLAG_TWO_STREAMS)):
             pl = db.plan(pod, flags=flags)
             ws = db.workspace(pl)
             pl.upload(ws, stream)
@@ -285,6 +293,7 @@ def run_sweep(args):
                          "prefill_TFLOPs": info.prefill_flops / (kern_us * 1e-6) / 1e12,
                          "error_word": db.error_word(pl, ws)}
         res["speedup_vs_sequential"] = res["sequential"]["step_us"] / res["fused"]["step_us"]
+        res["speedup_vs_two_streams"] = res["two_streams"]["step_us"] / res["fused"]["step_us"]
         res["peaks"] = peak_src
         print(json.dumps(res), flush=True)
         del db
@@ -382,6 +391,18 @@ def main():
     total_ms, kern_ms, (tw0, tw1) = timed_loop(fused, ws, args.steps, True)
     clocks = sampler.summary(tw0, tw1)
     seq_ms, seq_kern, _ = timed_loop(seq, ws_seq, max(50, args.steps // 4), True)
+    # ablations through the same API: the two kernels of the sequential path on two concurrent streams,
+    # and every CTA starting on one role (the proportional rule gives 1:1 with two CTAs per SM)
+    k_abl = max(50, args.steps // 4)
+    ablations = {}
+    for name, kw in (("two_streams", dict(flags=pod.POD_FLAG_TWO_STREAMS)),
+                     ("prefill_first_1_0", dict(ratio=(1, 0))), ("decode_first_0_1", dict(ratio=(0, 1)))):
+        pl_a = db.plan(pod, **kw)
+        ws_a = db.workspace(pl_a)
+        pl_a.upload(ws_a, stream)
+        a_ms, _, _ = timed_loop(pl_a, ws_a, k_abl, False)
+        ablations[name] = {"step_us": max_over_ranks(a_ms * 1e3 / k_abl), "error_word": db.error_word(pl_a, ws_a)}
+        del ws_a
     sampler.stop()
     err_word = db.error_word(fused, ws)
 
@@ -479,6 +500,9 @@ def main():
                      "traffic": traffic, "algorithmic_bytes": int(alg_bytes),
                      "algorithmic_flops_prefill": int(info.prefill_flops), "kernel_us": kern_us},
         "sequential_us": seq_us, "sequential_kernels_us": seq_kern_us, "speedup_vs_sequential": seq_us / us,
+        "ablations": dict(ablations, fused_step_us=us,
+                          note="two_streams = prefill-only and decode-only kernels on concurrent streams; "
+                               "x_first = ratio p:d forced so every CTA starts on that role"),
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
         "plan": {"prefill_items": info.num_prefill_items, "decode_items": info.num_decode_items,
                  "merge_items": info.num_merge_items, "chunk_pages": info.chunk_pages,

@@ -73,6 +73,10 @@ enum {
 #define POD_FLAG_SELFTEST_TIMEOUT 8u /* diagnostic: CTA 0 first waits (1 ms limit) on a barrier that
                                        nothing arrives at, so the wait expires and POD_ERR_TIMEOUT is
                                        recorded in the error word; the attention itself still runs */
+#define POD_FLAG_TWO_STREAMS 16u /* ablation: the prefill-only kernel on the caller's stream and the
+                                    decode-only kernel on a library-owned stream forked from it and
+                                    joined back with events (concurrent kernels, no co-location
+                                    control); ignored with POD_FLAG_SEQUENTIAL */
 
 typedef struct pod_attn_config {
   int32_t num_q_heads;      /* Hq */
@@ -144,7 +148,8 @@ int pod_attn_upload(const pod_attn_plan_t* plan, void* workspace, size_t workspa
 /* Enqueue one hybrid-batch attention on `stream`: reset the ticket, queue and
  * merge counters in the workspace, launch the persistent fused kernel (or, with
  * POD_FLAG_SEQUENTIAL in the plan's config, the prefill-only then decode-only
- * kernels).  Split-KV partials are merged by the warp that finishes a row's
+ * kernels; with POD_FLAG_TWO_STREAMS, the two on concurrent streams, the call
+ * still completing in `stream` order).  Split-KV partials are merged by the warp that finishes a row's
  * last split (a completion counter, no waiting), or, with POD_FLAG_MERGE_KERNEL,
  * by the LSE merge kernel launched afterwards.  Asynchronous.
  * q/k/v/o pointers: device, 16-byte aligned; unused sides (P == 0 or B == 0)

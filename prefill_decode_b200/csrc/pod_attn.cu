@@ -1006,6 +1006,33 @@ int configure_kernels() {
   return POD_OK;
 }
 
+// Library-owned side stream and fork/join events for the two-stream ablation,
+// one set per device, made on first use; `lock` serialises the enqueue order.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex lock;
+};
+
+int side_stream(SideStream** out) {
+  static SideStream sides[64];
+  static std::mutex make;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev >= 64) return POD_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(make);
+  SideStream& s = sides[dev];
+  if (!s.stream) {
+    e = cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  *out = &s;
+  return POD_OK;
+}
+
 template <int D>
 int launch(const pod_attn_plan_t* pl, PodParams& prm, const MergeParams& mp, cudaStream_t st) {
   int rc = configure_kernels<D>();
@@ -1024,6 +1051,24 @@ int launch(const pod_attn_plan_t* pl, PodParams& prm, const MergeParams& mp, cud
       prm.use_tmem = 0;
       pod_attn_kernel<D><<<pl->grid, kThreads, smem, st>>>(prm);
     }
+  } else if ((pl->cfg.flags & POD_FLAG_TWO_STREAMS) && pl->n_pre > 0 && pl->n_dec > 0) {
+    SideStream* side = nullptr;
+    rc = side_stream(&side);
+    if (rc != POD_OK) return rc;
+    std::lock_guard<std::mutex> g(side->lock);
+    cudaError_t e = cudaEventRecord(side->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+    if (e != cudaSuccess) return cuda_fail(e);
+    prm.mode = kPrefillOnly;
+    prm.use_tmem = 1;
+    const int grid = pl->n_pre < pl->grid ? pl->n_pre : pl->grid;
+    pod_attn_kernel<D><<<grid, kThreads, smem, st>>>(prm);
+    prm.mode = kDecodeOnly;
+    prm.use_tmem = 0;
+    pod_attn_kernel<D><<<pl->grid, kThreads, smem, side->stream>>>(prm);
+    e = cudaEventRecord(side->join, side->stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side->join, 0);
+    if (e != cudaSuccess) return cuda_fail(e);
   } else if (pl->n_pre > 0 || pl->n_dec > 0) {
     prm.mode = kFused;
     prm.use_tmem = pl->n_pre > 0 ? 1 : 0;
