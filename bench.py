@@ -177,10 +177,11 @@ def cpu_oracle_time(b, decode_reqs, prefill_rows):
     w = b.workload
     t0 = time.perf_counter()
     od = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, w.num_kv_heads,
-                         requests=decode_reqs) if len(decode_reqs) else None
+                         requests=decode_reqs, first_row=b.num_prefill) if len(decode_reqs) else None
     t1 = time.perf_counter()
-    op = A.attend_prefill(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_ctx, b.scale, w.num_kv_heads,
-                          rows=prefill_rows) if len(prefill_rows) else None
+    op = A.attend_prefill_batched(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_qo_lens,
+                                  b.prefill_kv_lens, b.scale, w.num_kv_heads,
+                                  rows=prefill_rows) if len(prefill_rows) else None
     t2 = time.perf_counter()
     return t1 - t0, t2 - t1, od, op
 
@@ -189,11 +190,17 @@ def extrapolate(b, decode_reqs, prefill_rows, t_dec, t_pre):
     """Scale sampled oracle time to the whole batch by keys visited."""
     L = b.decode_lens.astype(np.int64)
     dec_scale = float(L.sum()) / max(1.0, float(L[list(decode_reqs)].sum())) if len(decode_reqs) else 0.0
-    C, P = b.prefill_ctx, b.prefill_len
-    keys_all = sum(C + i + 1 for i in range(P))
-    keys_s = sum(C + int(i) + 1 for i in prefill_rows)
+    keys = prefill_row_keys(b)
+    keys_all = int(keys.sum())
+    keys_s = int(keys[list(prefill_rows)].sum()) if len(prefill_rows) else 0
     pre_scale = keys_all / keys_s if keys_s else 0.0
     return t_dec * dec_scale + t_pre * pre_scale
+
+
+def prefill_row_keys(b) -> np.ndarray:
+    """Keys each prefill row sees (C_i + i + 1 for row i of request i), over all requests in order."""
+    out = [np.arange(P, dtype=np.int64) + (K - P) + 1 for P, K in zip(b.prefill_qo_lens, b.prefill_kv_lens)]
+    return np.concatenate(out) if out else np.zeros(0, dtype=np.int64)
 
 
 def blas_threads() -> int:
@@ -206,7 +213,7 @@ def blas_threads() -> int:
 
 
 def sample_sets(b, frac_den: int):
-    B, P = b.workload.num_decode, b.prefill_len
+    B, P = b.workload.num_decode, b.workload.prefill_rows
     reqs = list(range(0, B, frac_den)) if B else []
     rows = list(range(0, P, frac_den)) if P else []
     return reqs, rows
@@ -242,6 +249,7 @@ def config_dict(w, b, mode):
     return {"workload": w.name, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "prefill_len": w.prefill_len, "prefill_ctx": w.prefill_ctx,
             "num_decode": w.num_decode, "decode_lens": f"{w.lens_kind}{list(w.lens_args)}, seed {w.seed}",
+            **({"prefill_requests": [list(r) for r in w.prefill_requests]} if w.prefill_reqs is not None else {}),
             "sum_decode_len": int(L.sum()) if len(L) else 0, "page_size": 16, "mode": mode,
             "l2": "no flush: inputs larger than L2 (the KV streamed per step exceeds 126 MB)"}
 

@@ -107,36 +107,59 @@ typedef struct pod_attn_plan_info {
   int32_t grid;               /* CTAs of the persistent kernel */
   int64_t workspace_bytes;
   int64_t error_offset;       /* byte offset of the int32 device error word */
-  int64_t prefill_flops;      /* 4 d Hq sum over chunk rows of keys seen */
+  int64_t prefill_flops;      /* 4 d Hq sum over every chunk row of the keys it sees */
   int64_t decode_flops;       /* 4 d Hq sum_r L_r */
-  int64_t kv_bytes;           /* 4 d Hkv (C + P + sum_r L_r): K and V read once */
-  int64_t qo_bytes;           /* 4 d Hq (P + B): Q read and O written once */
+  int64_t kv_bytes;           /* 4 d Hkv (sum_i (C_i + P_i) + sum_r L_r): K and V read once */
+  int64_t qo_bytes;           /* 4 d Hq (sum_i P_i + B): Q read and O written once */
   int64_t table_bytes;        /* bytes pod_attn_upload copies host -> device */
+  int32_t num_prefill_requests; /* NP: block-table / kv_lens rows 0..NP-1; decodes follow */
+  int32_t num_prefill_rows;     /* sum_i P_i: rows of q_prefill / o_prefill */
 } pod_attn_plan_info;
 
 /* Build the schedule for one hybrid batch on the host (no device work).
- * prefill_qo_len = P (0 = no prefill); prefill_kv_len = C + P (ignored if P == 0);
- * decode_kv_lens = host array of B lengths, each >= 1.  The work items, the
- * split-KV partition and the ticket ratio follow the rule documented in
- * oracle/plan_ref.py (the pages fix no formula).  On success *plan_out owns a
- * new plan and *workspace_bytes_out (nullable) receives the device workspace
- * size that pod_attn_upload / pod_attn_run need.
+ * One prefill request: prefill_qo_len = P (0 = no prefill); prefill_kv_len = C + P
+ * (ignored if P == 0); it owns block-table / kv_lens row 0 even when P == 0,
+ * and decode request r owns row 1 + r.  decode_kv_lens = host array of B
+ * lengths, each >= 1.  The work items, the split-KV partition and the ticket
+ * ratio follow the rule documented in oracle/plan_ref.py (the pages fix no
+ * formula).  On success *plan_out owns a new plan and *workspace_bytes_out
+ * (nullable) receives the device workspace size that pod_attn_upload /
+ * pod_attn_run need.  Same as pod_attn_plan_batched with one prefill request.
  * Errors: POD_ERR_INVALID_ARG, POD_ERR_UNSUPPORTED, POD_ERR_CUDA (num_sms == 0
  * and no device could be queried). */
 int pod_attn_plan(const pod_attn_config* cfg, int32_t prefill_qo_len, int32_t prefill_kv_len,
                   int32_t num_decode, const int32_t* decode_kv_lens,
                   pod_attn_plan_t** plan_out, size_t* workspace_bytes_out);
 
+/* Batched hybrid batch: num_prefill (0..4096) chunked-prefill requests and
+ * num_decode decodes in one fused launch (the FlashInfer PR "Limit kv split when
+ * prefill tokens <= 1536" times such a batched POD next to the one-prefill form).
+ * Prefill request i (host arrays, length num_prefill): P_i = prefill_qo_lens[i]
+ * query rows (0 allowed: the request has no work but keeps its row) over
+ * prefill_kv_lens[i] = C_i + P_i keys, causal bottom-right; it owns block-table
+ * / kv_lens row i, and its rows of q_prefill / o_prefill follow those of
+ * requests 0..i-1.  Decode request r owns row num_prefill + r.  Rule, outputs
+ * and errors as pod_attn_plan. */
+int pod_attn_plan_batched(const pod_attn_config* cfg, int32_t num_prefill, const int32_t* prefill_qo_lens,
+                          const int32_t* prefill_kv_lens, int32_t num_decode, const int32_t* decode_kv_lens,
+                          pod_attn_plan_t** plan_out, size_t* workspace_bytes_out);
+
 /* Copy the plan's summary into *info.  Errors: POD_ERR_INVALID_ARG (null). */
 int pod_attn_plan_get_info(const pod_attn_plan_t* plan, pod_attn_plan_info* info);
 
 /* Host copies of the work tables, for bit-exact checks; any pointer may be null.
- *   prefill_items int32 [num_prefill_items, 4]: q0, q_head, kv_end, partial (-1)
+ *   prefill_items int32 [num_prefill_items, 4]: q0 (row within its request), q_head,
+ *                                               kv_end, prefill request
  *   decode_items  int32 [num_decode_items, 8]:  r, kv_head, k0, k1, partial (-1 = unsplit),
  *                                               merge item (-1 = unsplit), splits of the row, 0
  *   merge_items   int32 [num_merge_items, 4]:   r, kv_head, first_partial, num_splits */
 int pod_attn_plan_tables(const pod_attn_plan_t* plan, int32_t* prefill_items,
                          int32_t* decode_items, int32_t* merge_items);
+
+/* Copy the prefill request table (host int32 [num_prefill_requests, 4]: first
+ * row of the request in q_prefill, P_i, C_i, 0) into `out` (nullable = skip).
+ * Errors: POD_ERR_INVALID_ARG (null plan). */
+int pod_attn_plan_prefill_requests(const pod_attn_plan_t* plan, int32_t* out);
 
 /* Enqueue on `stream` (a cudaStream_t; NULL = legacy default stream) the copy
  * of the plan's work tables into `workspace` (device, >= workspace_bytes,
@@ -152,8 +175,12 @@ int pod_attn_upload(const pod_attn_plan_t* plan, void* workspace, size_t workspa
  * still completing in `stream` order).  Split-KV partials are merged by the warp that finishes a row's
  * last split (a completion counter, no waiting), or, with POD_FLAG_MERGE_KERNEL,
  * by the LSE merge kernel launched afterwards.  Asynchronous.
- * q/k/v/o pointers: device, 16-byte aligned; unused sides (P == 0 or B == 0)
- * may be null.  num_blocks = pages in each cache pool.  trace (nullable, used
+ * q/k/v/o pointers: device, 16-byte aligned; q_prefill / o_prefill hold the
+ * prefill requests' rows one after another ([sum_i P_i, Hq, d]); unused sides
+ * (no prefill rows, or B == 0) may be null.  block_table (device int32, row
+ * stride block_table_stride) and kv_lens (device int32) have one row per
+ * request: prefill requests first, then decodes.  num_blocks = pages in each
+ * cache pool.  trace (nullable, used
  * with POD_FLAG_TRACE): int32 [num_prefill_items + num_decode_items, 4], zeroed
  * by the caller; entry = {smid, cta, home role (0 prefill, 1 decode), times run}.
  * Errors: POD_ERR_INVALID_ARG, POD_ERR_WORKSPACE, POD_ERR_CUDA (launch failed). */

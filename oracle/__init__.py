@@ -26,10 +26,11 @@ from .attention import (  # noqa: F401
     gather_tokens,
     attend_decode,
     attend_prefill,
+    attend_prefill_batched,
     attend_rows,
     attend_partial,
     lse_merge,
     attend_brute_decode,
     attend_brute_prefill,
 )
-from .plan_ref import plan_ref, PlanRef  # noqa: F401
+from .plan_ref import plan_ref, plan_ref_batched, PlanRef  # noqa: F401

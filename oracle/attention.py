@@ -66,8 +66,9 @@ def _as_f64(bits_or_f: np.ndarray) -> np.ndarray:
 
 
 def attend_decode(q_dec, k_pool, v_pool, block_table, kv_lens, scale: float, num_kv_heads: int,
-                  requests=None) -> np.ndarray:
-    """Decode attention.  q_dec [B, Hq, d]; row r+1 of block_table / kv_lens is request r.
+                  requests=None, first_row: int = 1) -> np.ndarray:
+    """Decode attention.  q_dec [B, Hq, d]; row first_row + r of block_table /
+    kv_lens is request r (the rows before it belong to the prefill requests).
 
     Returns float64 [B, Hq, d] (or [len(requests), Hq, d] for a subset)."""
     q = _as_f64(q_dec)
@@ -77,18 +78,18 @@ def attend_decode(q_dec, k_pool, v_pool, block_table, kv_lens, scale: float, num
     reqs = range(B) if requests is None else list(requests)
     out = np.empty((len(reqs), Hq, d), dtype=np.float64)
     for o, r in enumerate(reqs):
-        L = int(kv_lens[1 + r])
+        L = int(kv_lens[first_row + r])
         for kvh in range(num_kv_heads):
-            K = gather_tokens(kp, block_table[1 + r], L, kvh)
-            V = gather_tokens(vp, block_table[1 + r], L, kvh)
+            K = gather_tokens(kp, block_table[first_row + r], L, kvh)
+            V = gather_tokens(vp, block_table[first_row + r], L, kvh)
             hs = slice(kvh * g, (kvh + 1) * g)
             out[o, hs] = attend_rows(q[r, hs], K, V, scale, [L] * g)
     return out
 
 
 def attend_prefill(q_pre, k_pool, v_pool, block_table, prior_ctx: int, scale: float, num_kv_heads: int,
-                   rows=None) -> np.ndarray:
-    """Causal chunked-prefill attention for request 0 (block_table row 0).
+                   rows=None, bt_row: int = 0) -> np.ndarray:
+    """Causal chunked-prefill attention for the request in block_table row bt_row.
 
     q_pre [P, Hq, d]; chunk row i sees keys 0..C+i.  Returns float64 [P, Hq, d]
     (or [len(rows), Hq, d] for a subset of chunk rows)."""
@@ -104,11 +105,36 @@ def attend_prefill(q_pre, k_pool, v_pool, block_table, prior_ctx: int, scale: fl
     L = C + int(sel.max()) + 1
     limits = C + sel + 1
     for kvh in range(num_kv_heads):
-        K = gather_tokens(kp, block_table[0], L, kvh)
-        V = gather_tokens(vp, block_table[0], L, kvh)
+        K = gather_tokens(kp, block_table[bt_row], L, kvh)
+        V = gather_tokens(vp, block_table[bt_row], L, kvh)
         for hh in range(g):
             h = kvh * g + hh
             out[:, h] = attend_rows(q[sel, h], K, V, scale, limits)
+    return out
+
+
+def attend_prefill_batched(q_pre, k_pool, v_pool, block_table, qo_lens, kv_lens, scale: float,
+                           num_kv_heads: int, rows=None) -> np.ndarray:
+    """Several chunked-prefill requests in one hybrid batch (the FlashInfer PR
+    "Limit kv split when prefill tokens <= 1536" times such a "Batched POD
+    Attention" next to the one-prefill POD): request i owns block_table row i, its P_i = qo_lens[i] query
+    rows follow those of requests 0..i-1 in q_pre [sum P_i, Hq, d], and its chunk
+    continues C_i = kv_lens[i] - P_i earlier tokens.  Each request is the single
+    chunked prefill above.  Returns float64 [sum P_i, Hq, d] (or the rows listed,
+    indexed into the concatenation)."""
+    q = _as_f64(q_pre)
+    total, Hq, d = q.shape
+    sel = np.arange(total) if rows is None else np.asarray(list(rows), dtype=np.int64)
+    out = np.empty((len(sel), Hq, d), dtype=np.float64)
+    start = 0
+    for i, (P, KV) in enumerate(zip(qo_lens, kv_lens)):
+        P, KV = int(P), int(KV)
+        mine = (sel >= start) & (sel < start + P)
+        if mine.any():
+            local = sel[mine] - start
+            out[mine] = attend_prefill(q[start:start + P], k_pool, v_pool, block_table, KV - P, scale,
+                                       num_kv_heads, rows=local, bt_row=i)
+        start += P
     return out
 
 
@@ -159,23 +185,25 @@ def _token(pool, bt_row, j, kvh):
     return [float(x) for x in pool[int(bt_row[j // PAGE]), kvh, j % PAGE, :]]
 
 
-def attend_brute_decode(q_dec, k_pool, v_pool, block_table, kv_lens, scale: float, num_kv_heads: int) -> np.ndarray:
+def attend_brute_decode(q_dec, k_pool, v_pool, block_table, kv_lens, scale: float, num_kv_heads: int,
+                        first_row: int = 1) -> np.ndarray:
     q = _as_f64(q_dec)
     kp, vp = _as_f64(k_pool), _as_f64(v_pool)
     B, Hq, d = q.shape
     g = Hq // num_kv_heads
     out = np.zeros((B, Hq, d))
     for r in range(B):
-        L = int(kv_lens[1 + r])
+        L = int(kv_lens[first_row + r])
         for h in range(Hq):
             kvh = h // g
-            keys = [_token(kp, block_table[1 + r], j, kvh) for j in range(L)]
-            vals = [_token(vp, block_table[1 + r], j, kvh) for j in range(L)]
+            keys = [_token(kp, block_table[first_row + r], j, kvh) for j in range(L)]
+            vals = [_token(vp, block_table[first_row + r], j, kvh) for j in range(L)]
             out[r, h] = _brute_one([float(x) for x in q[r, h]], keys, vals, scale)
     return out
 
 
-def attend_brute_prefill(q_pre, k_pool, v_pool, block_table, prior_ctx: int, scale: float, num_kv_heads: int) -> np.ndarray:
+def attend_brute_prefill(q_pre, k_pool, v_pool, block_table, prior_ctx: int, scale: float, num_kv_heads: int,
+                         bt_row: int = 0) -> np.ndarray:
     q = _as_f64(q_pre)
     kp, vp = _as_f64(k_pool), _as_f64(v_pool)
     P, Hq, d = q.shape
@@ -185,7 +213,7 @@ def attend_brute_prefill(q_pre, k_pool, v_pool, block_table, prior_ctx: int, sca
         for h in range(Hq):
             kvh = h // g
             n = prior_ctx + i + 1
-            keys = [_token(kp, block_table[0], j, kvh) for j in range(n)]
-            vals = [_token(vp, block_table[0], j, kvh) for j in range(n)]
+            keys = [_token(kp, block_table[bt_row], j, kvh) for j in range(n)]
+            vals = [_token(vp, block_table[bt_row], j, kvh) for j in range(n)]
             out[i, h] = _brute_one([float(x) for x in q[i, h]], keys, vals, scale)
     return out

@@ -14,13 +14,18 @@ Rule
     max_waves >= 0 (0 = 2); min_chunk_pages >= 0 (0 = 16); P >= 0;
     if P > 0: P <= prefill_kv_len <= 2^24; 0 <= B <= 65536; 1 <= L_r <= 2^24;
     sum_r L_r <= 2^31 - 1.
-  Prefill items (one 128-row query tile of one query head each), longest first:
-    for t = T-1 .. 0 (T = ceil(P/128)), for h = 0 .. Hq-1:
-      (q0 = 128 t, h, kv_end = C + min(128 (t+1), P), partial = -1).
+  Prefill requests i = 0 .. NP-1 (chunk P_i over C_i = kv_i - P_i earlier
+    tokens; the one-prefill form is NP = 1, P_0 = P).  Prefill items (one
+    128-row query tile of one query head each): for i, for t = T_i-1 .. 0
+    (T_i = ceil(P_i/128)), for h = 0 .. Hq-1: (q0 = 128 t, h,
+    kv_end = C_i + min(128 (t+1), P_i), request i); then stably sorted by
+    kv_end, longest first.  Prefill request table (q_start_i = P_0 + .. +
+    P_{i-1}, P_i, C_i, 0).
   Decode split: W = num_sms * ctas_per_sm * 4 decode warps; cap = max_waves * W;
     pages_r = ceil(L_r / 16); N = Hkv * sum pages_r; maxp = max pages_r;
     c = max(min_chunk_pages, ceil(N / cap)); then c += 1 while c < maxp and
-    Hkv * sum ceil(pages_r / c) > cap.  Request r is cut into
+    Hkv * sum ceil(pages_r / c) > cap.  Decode request r (block-table row
+    NP + r) is cut into
     S_r = ceil(pages_r / c) splits; split s covers pages
     [floor(s pages_r / S_r), floor((s+1) pages_r / S_r)), i.e. tokens
     [16 p0, min(16 p1, L_r)).
@@ -32,7 +37,7 @@ Rule
   Ratio p:d of per-SM tickets (ticket t -> prefill iff t mod (p+d) < p):
     explicit (ratio_p, ratio_d) reduced by gcd (a zero side gives 1:0 or 0:1);
     proportional (both 0): no prefill -> 0:1; no decode -> 1:0; otherwise
-    cost_pre = 4 d sum over prefill rows of keys seen, times Hq (FLOPs);
+    cost_pre = 4 d sum over every prefill request's rows of keys seen, times Hq (FLOPs);
     cost_dec = 248 * 4 d Hkv sum_r L_r (bytes x 248, the measured B200
     tensor-FLOP/s per HBM-byte/s); k = ctas_per_sm;
     n_p = floor((2 k cost_pre + tot) / (2 tot)), tot = cost_pre + cost_dec,
@@ -52,6 +57,7 @@ BM = 128
 WARPS_PER_CTA = 4
 COST_RATIO = 248
 MAX_SMS = 512
+MAX_PREFILL_REQUESTS = 4096
 
 
 class PlanError(ValueError):
@@ -60,7 +66,7 @@ class PlanError(ValueError):
 
 @dataclasses.dataclass
 class PlanRef:
-    prefill_items: np.ndarray   # int32 [n, 4]
+    prefill_items: np.ndarray   # int32 [n, 4]: q0, q head, kv_end, request
     decode_items: np.ndarray    # int32 [n, 8]
     merge_items: np.ndarray     # int32 [n, 4]
     ctas_per_sm: int
@@ -68,6 +74,7 @@ class PlanRef:
     ratio_d: int
     chunk_pages: int
     num_partials: int
+    prefill_requests: np.ndarray = None   # int32 [NP, 4]: q_start, P, C, 0
 
 
 def _ceil(a: int, b: int) -> int:
@@ -75,11 +82,20 @@ def _ceil(a: int, b: int) -> int:
 
 
 def plan_ref(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
-             prefill_len: int, prefill_kv_len: int, decode_lens: Sequence[int], *,
-             page_size: int = 16, ctas_per_sm: int = 0, ratio_p: int = 0, ratio_d: int = 0,
-             max_waves: int = 0, min_chunk_pages: int = 0) -> PlanRef:
+             prefill_len: int, prefill_kv_len: int, decode_lens: Sequence[int], **knobs) -> PlanRef:
+    """One prefill request (block-table row 0, P = 0 for none) and B decodes (rows 1..B)."""
+    return plan_ref_batched(num_q_heads, num_kv_heads, head_dim, num_sms, [prefill_len], [prefill_kv_len],
+                            decode_lens, **knobs)
+
+
+def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
+                     prefill_qo_lens: Sequence[int], prefill_kv_lens: Sequence[int], decode_lens: Sequence[int], *,
+                     page_size: int = 16, ctas_per_sm: int = 0, ratio_p: int = 0, ratio_d: int = 0,
+                     max_waves: int = 0, min_chunk_pages: int = 0) -> PlanRef:
+    """NP prefill requests (block-table rows 0..NP-1) and B decodes (rows NP..NP+B-1)."""
     Hq, Hkv, d = int(num_q_heads), int(num_kv_heads), int(head_dim)
-    P, KVp = int(prefill_len), int(prefill_kv_len)
+    pre_qo = [int(x) for x in prefill_qo_lens]
+    pre_kv = [int(x) for x in prefill_kv_lens]
     lens = [int(x) for x in decode_lens]
     B = len(lens)
     if Hq <= 0 or Hkv <= 0 or Hq % Hkv:
@@ -91,21 +107,31 @@ def plan_ref(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
         raise PlanError("invalid launch knobs")
     if ratio_p < 0 or ratio_d < 0 or max_waves < 0 or min_chunk_pages < 0:
         raise PlanError("invalid knobs")
-    if P < 0 or (P > 0 and not (P <= KVp <= (1 << 24))):
+    if len(pre_qo) != len(pre_kv) or len(pre_qo) > MAX_PREFILL_REQUESTS:
+        raise PlanError("invalid prefill requests")
+    for P, KVp in zip(pre_qo, pre_kv):
+        if P < 0 or (P > 0 and not (P <= KVp <= (1 << 24))):
+            raise PlanError("invalid prefill lengths")
+    if sum(pre_qo) > (1 << 24):
         raise PlanError("invalid prefill lengths")
     if B > 65536 or any(not (1 <= L <= (1 << 24)) for L in lens) or sum(lens) > (1 << 31) - 1:
         raise PlanError("invalid decode lengths")
     k = 2 if ctas_per_sm == 0 else ctas_per_sm
     waves = 2 if max_waves == 0 else max_waves
     minc = 16 if min_chunk_pages == 0 else min_chunk_pages
-    C = KVp - P if P > 0 else 0
+    ctx = [KVp - P if P > 0 else 0 for P, KVp in zip(pre_qo, pre_kv)]
 
-    # prefill items, longest (last) tile first
+    # prefill items per request, last tile first; then all requests' items longest first
     pre = []
-    T = _ceil(P, BM)
-    for t in range(T - 1, -1, -1):
-        for h in range(Hq):
-            pre.append((BM * t, h, C + min(BM * (t + 1), P), -1))
+    for i, (P, C) in enumerate(zip(pre_qo, ctx)):
+        for t in range(_ceil(P, BM) - 1, -1, -1):
+            for h in range(Hq):
+                pre.append((BM * t, h, C + min(BM * (t + 1), P), i))
+    pre.sort(key=lambda e: -e[2])          # stable: equal kv_end keep (request, tile, head) order
+    preq, q_start = [], 0
+    for P, C in zip(pre_qo, ctx):
+        preq.append((q_start, P, C, 0))
+        q_start += P
 
     # decode split
     W = num_sms * k * WARPS_PER_CTA
@@ -152,10 +178,11 @@ def plan_ref(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
         p_, d_ = 1, 0
     else:
         rows_keys = 0
-        for t in range(T):
-            q0 = BM * t
-            n = min(BM, P - q0)
-            rows_keys += n * (C + 1) + n * q0 + n * (n - 1) // 2
+        for P, C in zip(pre_qo, ctx):
+            for t in range(_ceil(P, BM)):
+                q0 = BM * t
+                n = min(BM, P - q0)
+                rows_keys += n * (C + 1) + n * q0 + n * (n - 1) // 2
         cost_pre = 4 * d * Hq * rows_keys
         cost_dec = COST_RATIO * 4 * d * Hkv * sum(lens)
         tot = cost_pre + cost_dec
@@ -175,4 +202,4 @@ def plan_ref(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
         a = np.asarray(rows, dtype=np.int32)
         return a.reshape(len(rows), w)
 
-    return PlanRef(arr(pre, 4), arr([e[4] for e in dec], 8), arr(merge, 4), k, p_, d_, c, npart)
+    return PlanRef(arr(pre, 4), arr([e[4] for e in dec], 8), arr(merge, 4), k, p_, d_, c, npart, arr(preq, 4))

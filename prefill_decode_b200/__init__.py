@@ -35,6 +35,7 @@ EXPORTED = [
     "pod_attn_plan", "pod_attn_plan_get_info", "pod_attn_plan_tables", "pod_attn_upload", "pod_attn_run",
     "pod_attn_plan_set_events", "pod_attn_event_create", "pod_attn_event_destroy", "pod_attn_event_elapsed_ms",
     "pod_attn_plan_destroy", "pod_attn_status_string", "pod_attn_last_cuda_error", "pod_attn_run_static",
+    "pod_attn_plan_batched", "pod_attn_plan_prefill_requests",
 ]
 
 
@@ -48,7 +49,8 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_prefill_items", "num_decode_items", "num_merge_items", "num_partials", "ctas_per_sm",
         "ratio_prefill", "ratio_decode", "chunk_pages", "num_sms", "grid")] + [(n, ctypes.c_int64) for n in (
-            "workspace_bytes", "error_offset", "prefill_flops", "decode_flops", "kv_bytes", "qo_bytes", "table_bytes")]
+            "workspace_bytes", "error_offset", "prefill_flops", "decode_flops", "kv_bytes", "qo_bytes", "table_bytes")] + [
+            (n, ctypes.c_int32) for n in ("num_prefill_requests", "num_prefill_rows")]
 
 
 class PodError(RuntimeError):
@@ -71,6 +73,9 @@ def lib() -> ctypes.CDLL:
         vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
         L.pod_attn_plan.argtypes = [ctypes.POINTER(Config), i32, i32, i32, ctypes.POINTER(i32),
                                     ctypes.POINTER(vp), ctypes.POINTER(sz)]
+        L.pod_attn_plan_batched.argtypes = [ctypes.POINTER(Config), i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                            i32, ctypes.POINTER(i32), ctypes.POINTER(vp), ctypes.POINTER(sz)]
+        L.pod_attn_plan_prefill_requests.argtypes = [vp, vp]
         L.pod_attn_plan_get_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
         L.pod_attn_plan_tables.argtypes = [vp, vp, vp, vp]
         L.pod_attn_upload.argtypes = [vp, vp, sz, vp]
@@ -120,10 +125,13 @@ def _stream(stream) -> Optional[int]:
 
 
 class Plan:
-    """Host-side schedule of one hybrid batch (``pod_attn_plan``)."""
+    """Host-side schedule of one hybrid batch.  ``prefill_len`` / ``prefill_kv_len``
+    are ints for one prefill request (``pod_attn_plan``: block-table row 0,
+    decodes from row 1) or equal-length sequences for several
+    (``pod_attn_plan_batched``: rows 0..NP-1, decodes from row NP)."""
 
-    def __init__(self, num_q_heads: int, num_kv_heads: int, head_dim: int, prefill_len: int,
-                 prefill_kv_len: int, decode_lens: Sequence[int], *, num_sms: int = 0,
+    def __init__(self, num_q_heads: int, num_kv_heads: int, head_dim: int, prefill_len,
+                 prefill_kv_len, decode_lens: Sequence[int], *, num_sms: int = 0,
                  ctas_per_sm: int = 0, ratio: Tuple[int, int] = (0, 0), max_waves: int = 0,
                  min_chunk_pages: int = 0, flags: int = 0, page_size: int = 16):
         L = lib()
@@ -134,8 +142,19 @@ class Plan:
         h = ctypes.c_void_p()
         ws = ctypes.c_size_t()
         lp = lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) if lens.size else None
-        _check(L.pod_attn_plan(ctypes.byref(self.cfg), int(prefill_len), int(prefill_kv_len), int(lens.size),
-                               lp, ctypes.byref(h), ctypes.byref(ws)), "pod_attn_plan")
+        if np.ndim(prefill_len) == 0:
+            _check(L.pod_attn_plan(ctypes.byref(self.cfg), int(prefill_len), int(prefill_kv_len), int(lens.size),
+                                   lp, ctypes.byref(h), ctypes.byref(ws)), "pod_attn_plan")
+        else:
+            qo = np.ascontiguousarray(np.asarray(prefill_len, dtype=np.int32))
+            kv = np.ascontiguousarray(np.asarray(prefill_kv_len, dtype=np.int32))
+            if qo.shape != kv.shape:
+                raise ValueError("prefill_len and prefill_kv_len differ in length")
+            self._pre = (qo, kv)
+            qp = qo.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) if qo.size else None
+            kp = kv.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) if kv.size else None
+            _check(L.pod_attn_plan_batched(ctypes.byref(self.cfg), int(qo.size), qp, kp, int(lens.size), lp,
+                                           ctypes.byref(h), ctypes.byref(ws)), "pod_attn_plan_batched")
         self._h = h
         self.workspace_bytes = int(ws.value)
         self.info = PlanInfo()
@@ -150,6 +169,12 @@ class Plan:
     @property
     def handle(self) -> ctypes.c_void_p:
         return self._h
+
+    def prefill_requests(self) -> np.ndarray:
+        """int32 [NP, 4]: first row in q_prefill, P_i, C_i, 0."""
+        out = np.zeros((self.info.num_prefill_requests, 4), dtype=np.int32)
+        _check(lib().pod_attn_plan_prefill_requests(self._h, out.ctypes.data), "pod_attn_plan_prefill_requests")
+        return out
 
     def tables(self):
         i = self.info

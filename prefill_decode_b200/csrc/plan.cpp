@@ -25,8 +25,8 @@ struct DecEntry {
 
 }  // namespace
 
-int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t kv_len_prefill,
-                   int32_t B, const int32_t* lens, pod_attn_plan_t** out) {
+int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const int32_t* pre_qo,
+                   const int32_t* pre_kv, int32_t B, const int32_t* lens, pod_attn_plan_t** out) {
   using namespace pod;
   if (!cfg || !out) return POD_ERR_INVALID_ARG;
   const int32_t Hq = cfg->num_q_heads, Hkv = cfg->num_kv_heads, d = cfg->head_dim;
@@ -37,7 +37,14 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t k
   if (cfg->ctas_per_sm < 0 || cfg->ctas_per_sm > 2) return POD_ERR_INVALID_ARG;
   if (cfg->ratio_prefill < 0 || cfg->ratio_decode < 0 || cfg->max_waves < 0 || cfg->min_chunk_pages < 0)
     return POD_ERR_INVALID_ARG;
-  if (P < 0 || (P > 0 && (kv_len_prefill < P || kv_len_prefill > (1 << 24)))) return POD_ERR_INVALID_ARG;
+  if (NP < 0 || NP > kMaxPrefillRequests || (NP > 0 && (!pre_qo || !pre_kv))) return POD_ERR_INVALID_ARG;
+  int64_t sumP = 0;
+  for (int32_t i = 0; i < NP; ++i) {
+    const int32_t P = pre_qo[i];
+    if (P < 0 || (P > 0 && (pre_kv[i] < P || pre_kv[i] > (1 << 24)))) return POD_ERR_INVALID_ARG;
+    sumP += P;
+  }
+  if (sumP > (1 << 24)) return POD_ERR_INVALID_ARG;
   if (B < 0 || B > 65536 || (B > 0 && !lens)) return POD_ERR_INVALID_ARG;
   int64_t sumL = 0;
   for (int32_t r = 0; r < B; ++r) {
@@ -52,9 +59,10 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t k
   const int32_t k = cfg->ctas_per_sm == 0 ? 2 : cfg->ctas_per_sm;
   const int32_t waves = cfg->max_waves == 0 ? 2 : cfg->max_waves;
   const int32_t minc = cfg->min_chunk_pages == 0 ? 16 : cfg->min_chunk_pages;
-  const int32_t C = P > 0 ? kv_len_prefill - P : 0;
-  pl->P = P;
-  pl->C = C;
+  std::vector<int32_t> ctx(NP);
+  for (int32_t i = 0; i < NP; ++i) ctx[i] = pre_qo[i] > 0 ? pre_kv[i] - pre_qo[i] : 0;
+  pl->NP = NP;
+  pl->P = (int32_t)sumP;
   pl->B = B;
   pl->g = g;
   pl->ctas = k;
@@ -62,14 +70,27 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t k
   pl->grid = num_sms * k;
   pl->decode_lens.assign(lens, lens + B);
 
-  // ---- prefill items: one 128-row query tile of one query head, last tile first
-  const int32_t T = (int32_t)ceil_div(P, kBM);
-  for (int32_t t = T - 1; t >= 0; --t)
-    for (int32_t h = 0; h < Hq; ++h) {
-      int32_t item[kPrefillItemInts] = {kBM * t, h, C + std::min(kBM * (t + 1), P), -1};
-      pl->pre.insert(pl->pre.end(), item, item + kPrefillItemInts);
-    }
-  pl->n_pre = T * Hq;
+  // ---- prefill items: one 128-row query tile of one query head, per request last
+  // tile first, then all requests' items longest (largest kv_end) first, stably
+  struct PreEntry {
+    int32_t item[kPrefillItemInts];
+  };
+  std::vector<PreEntry> pents;
+  for (int32_t i = 0; i < NP; ++i) {
+    const int32_t P = pre_qo[i], C = ctx[i];
+    for (int32_t t = (int32_t)ceil_div(P, kBM) - 1; t >= 0; --t)
+      for (int32_t h = 0; h < Hq; ++h) pents.push_back(PreEntry{{kBM * t, h, C + std::min(kBM * (t + 1), P), i}});
+  }
+  std::stable_sort(pents.begin(), pents.end(),
+                   [](const PreEntry& a, const PreEntry& b) { return a.item[2] > b.item[2]; });
+  for (const PreEntry& e : pents) pl->pre.insert(pl->pre.end(), e.item, e.item + kPrefillItemInts);
+  pl->n_pre = (int32_t)pents.size();
+  int32_t q_start = 0;
+  for (int32_t i = 0; i < NP; ++i) {
+    const int32_t rq[kPrefillReqInts] = {q_start, pre_qo[i], ctx[i], 0};
+    pl->preq.insert(pl->preq.end(), rq, rq + kPrefillReqInts);
+    q_start += pre_qo[i];
+  }
 
   // ---- decode split: chunk c pages, at most waves x decode warps items
   const int64_t W = (int64_t)num_sms * k * kWarpsPerCta;
@@ -125,15 +146,19 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t k
   pl->n_part = npart;
 
   // ---- algorithmic work (roofline numerators)
-  int64_t rows_keys = 0;
-  for (int32_t t = 0; t < T; ++t) {
-    const int64_t q0 = (int64_t)kBM * t, n = std::min<int64_t>(kBM, P - q0);
-    rows_keys += n * (C + 1) + n * q0 + n * (n - 1) / 2;
+  int64_t rows_keys = 0, pre_kv_tokens = 0;
+  for (int32_t i = 0; i < NP; ++i) {
+    const int64_t P = pre_qo[i], C = ctx[i];
+    for (int64_t q0 = 0; q0 < P; q0 += kBM) {
+      const int64_t n = std::min<int64_t>(kBM, P - q0);
+      rows_keys += n * (C + 1) + n * q0 + n * (n - 1) / 2;
+    }
+    if (P > 0) pre_kv_tokens += C + P;
   }
   pl->prefill_flops = 4LL * d * Hq * rows_keys;
   pl->decode_flops = 4LL * d * Hq * sumL;
-  pl->kv_bytes = 4LL * d * Hkv * ((P > 0 ? (int64_t)C + P : 0) + sumL);
-  pl->qo_bytes = 4LL * d * Hq * ((int64_t)P + B);
+  pl->kv_bytes = 4LL * d * Hkv * (pre_kv_tokens + sumL);
+  pl->qo_bytes = 4LL * d * Hq * (sumP + B);
 
   // ---- ticket ratio p:d
   int32_t rp, rd;
@@ -176,7 +201,8 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t k
   pl->off_pre = align_up(pl->off_merge_cnt + 4LL * pl->n_merge, 256);
   pl->off_dec = align_up(pl->off_pre + 4LL * kPrefillItemInts * pl->n_pre, 256);
   pl->off_merge = align_up(pl->off_dec + 4LL * kDecodeItemInts * pl->n_dec, 256);
-  pl->off_part_o = align_up(pl->off_merge + 4LL * kMergeItemInts * pl->n_merge, 256);
+  pl->off_preq = align_up(pl->off_merge + 4LL * kMergeItemInts * pl->n_merge, 256);
+  pl->off_part_o = align_up(pl->off_preq + 4LL * kPrefillReqInts * NP, 256);
   pl->off_part_lse = align_up(pl->off_part_o + 4LL * g * d * npart, 256);
   pl->ws_bytes = align_up(pl->off_part_lse + 4LL * g * npart, 256);
   pl->image.assign((size_t)(pl->off_part_o - kCountersBytes), 0);
@@ -186,6 +212,8 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t k
     std::memcpy(pl->image.data() + (pl->off_dec - kCountersBytes), pl->dec.data(), pl->dec.size() * 4);
   if (!pl->merge.empty())
     std::memcpy(pl->image.data() + (pl->off_merge - kCountersBytes), pl->merge.data(), pl->merge.size() * 4);
+  if (!pl->preq.empty())
+    std::memcpy(pl->image.data() + (pl->off_preq - kCountersBytes), pl->preq.data(), pl->preq.size() * 4);
   *out = pl;
   return POD_OK;
 }

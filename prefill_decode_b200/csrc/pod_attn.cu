@@ -57,6 +57,7 @@ struct alignas(64) PodParams {
   const int4* pre_items;
   const int4* dec_items;   // two int4 per item
   const int4* merge_items; // r, kvh, first_partial, num_splits
+  const int4* pre_reqs;    // per prefill request: first row in q_pre / o_pre, P, C, 0
   int32_t* merge_cnt;      // splits finished per merge item (zero at launch)
   float* part_o;
   float* part_lse;
@@ -65,7 +66,7 @@ struct alignas(64) PodParams {
   int32_t kv_rows;         // num_blocks * Hkv * 16 (rows of the K/V tensor maps)
   int32_t num_blocks;
   int32_t n_pre, n_dec;
-  int32_t Hq, Hkv, g, P, C, B;
+  int32_t Hq, Hkv, g, NP, B;   // NP prefill requests own block-table rows 0..NP-1
   int32_t ratio_p, ratio_d;
   int32_t mode;
   int32_t use_tmem;
@@ -159,9 +160,9 @@ struct PageWindows {
   int cur, nxt, w;
 };
 
-__device__ __forceinline__ int load_page_window(const PodParams& p, int w, int kv_end, int lane) {
+__device__ __forceinline__ int load_page_window(const PodParams& p, const int* bt_row, int w, int kv_end, int lane) {
   const int gp = 32 * w + lane;
-  return gp * kPage < kv_end ? __ldg(&p.block_table[gp]) : 0;
+  return gp * kPage < kv_end ? __ldg(&bt_row[gp]) : 0;
 }
 
 // Tensor-map row of page `lane & 3` of key tile kb (kb in window w or w + 1);
@@ -215,12 +216,13 @@ template <int D>
 __device__ bool prefill_tma(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t t0) {
   using CF = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  const int qh = it.y, kv_end = it.z;
+  const int qh = it.y, kv_end = it.z, req = it.w;
   const int kvh = qh / p.g;
   const int nkb = (kv_end + kBN - 1) / kBN;
   const PrefillSmem<D> sm{smem};
-  if (lane == 0 && p.kv_lens && __ldg(&p.kv_lens[0]) < kv_end) record_error(p, POD_ERR_PLAN_MISMATCH, 0);
-  PageWindows pw{load_page_window(p, 0, kv_end, lane), load_page_window(p, 1, kv_end, lane), 0};
+  const int* bt_row = p.block_table + (size_t)req * p.bt_stride;
+  if (lane == 0 && p.kv_lens && __ldg(&p.kv_lens[req]) < kv_end) record_error(p, POD_ERR_PLAN_MISMATCH, req);
+  PageWindows pw{load_page_window(p, bt_row, 0, kv_end, lane), load_page_window(p, bt_row, 1, kv_end, lane), 0};
   for (int j = 0; j < nkb && j < CF::kKSlots; ++j) {
     const uint32_t t = t0 + j;
     const int r = tile_page_row(p, pw, j, kvh, kv_end, lane);
@@ -232,7 +234,7 @@ __device__ bool prefill_tma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
     if (((j + CF::kVSlots) >> 3) > pw.w) {   // tile j+2 enters the next window; fetch the one after it
       ++pw.w;
       pw.cur = pw.nxt;
-      pw.nxt = load_page_window(p, pw.w + 1, kv_end, lane);
+      pw.nxt = load_page_window(p, bt_row, pw.w + 1, kv_end, lane);
     }
     const bool more_k = j + CF::kKSlots < nkb;
     const int rk = more_k ? tile_page_row(p, pw, j + CF::kKSlots, kvh, kv_end, lane) : 0;
@@ -345,22 +347,24 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
                                 uint32_t t0, uint32_t nq) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q0 = it.x, qh = it.y, kv_end = it.z;
+  const int4 rq = __ldg(&p.pre_reqs[it.w]);       // first row in q_pre / o_pre, P, C
+  const int q_first = rq.x, P = rq.y, C = rq.z;
   const int nkb = (kv_end + kBN - 1) / kBN;
   const int row = tid;
-  const int row_limit = min(p.C + q0 + row + 1, kv_end);
-  const int full_tiles = (p.C + q0 + 1) / kBN;   // tiles visible to every row of this item
+  const int row_limit = min(C + q0 + row + 1, kv_end);
+  const int full_tiles = (C + q0 + 1) / kBN;     // tiles visible to every row of this item
   const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
   const float sl2 = p.scale_log2;
   {
     // Q row (bf16 pairs along d) into TMEM lane `row`; rows past the chunk are zero
     const int q = q0 + row;
-    const uint4* src = reinterpret_cast<const uint4*>(p.q_pre + ((size_t)q * p.Hq + qh) * D);
+    const uint4* src = reinterpret_cast<const uint4*>(p.q_pre + ((size_t)(q_first + q) * p.Hq + qh) * D);
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const uint4 v = q < p.P ? __ldg(src + c * 8 + i) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 v = q < P ? __ldg(src + c * 8 + i) : make_uint4(0u, 0u, 0u, 0u);
         w[4 * i] = v.x;
         w[4 * i + 1] = v.y;
         w[4 * i + 2] = v.z;
@@ -464,8 +468,8 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
     float o[32];
     tmem_ld32(tmem + t_lane + kTmemO + c * 32, o);
     tmem_wait_ld();
-    if (q < p.P) {
-      uint4* dst = reinterpret_cast<uint4*>(p.o_pre + ((size_t)q * p.Hq + qh) * D + c * 32);
+    if (q < P) {
+      uint4* dst = reinterpret_cast<uint4*>(p.o_pre + ((size_t)(q_first + q) * p.Hq + qh) * D + c * 32);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         uint4 v;
@@ -629,10 +633,10 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
     const int np = (k1 - k0 + kPage - 1) / kPage;
     // block ids: bt_cur holds pages [32 win, 32 win + 32) of the item, bt_nxt the next window;
     // the request's length is read in the same round trip and checked once the pages are under way
-    const int* bt_item = p.block_table + (size_t)(1 + r) * p.bt_stride + p0;
+    const int* bt_item = p.block_table + (size_t)(p.NP + r) * p.bt_stride + p0;
     int bt_cur = lane < np ? __ldg(bt_item + lane) : 0;
     int bt_nxt = 32 + lane < np ? __ldg(bt_item + 32 + lane) : 0;
-    const int len_now = (lane == 0 && p.kv_lens) ? __ldg(&p.kv_lens[1 + r]) : k1;
+    const int len_now = (lane == 0 && p.kv_lens) ? __ldg(&p.kv_lens[p.NP + r]) : k1;
     int win = 0;
     {
       const int pre = np < CF::kNS ? np : CF::kNS;
@@ -1102,8 +1106,9 @@ const char* pod_attn_status_string(int s) {
 
 int pod_attn_last_cuda_error(void) { return g_last_cuda; }
 
-int pod_attn_plan(const pod_attn_config* cfg, int32_t prefill_qo_len, int32_t prefill_kv_len, int32_t num_decode,
-                  const int32_t* decode_kv_lens, pod_attn_plan_t** plan_out, size_t* workspace_bytes_out) {
+int pod_attn_plan_batched(const pod_attn_config* cfg, int32_t num_prefill, const int32_t* prefill_qo_lens,
+                          const int32_t* prefill_kv_lens, int32_t num_decode, const int32_t* decode_kv_lens,
+                          pod_attn_plan_t** plan_out, size_t* workspace_bytes_out) {
   if (!cfg || !plan_out) return POD_ERR_INVALID_ARG;
   *plan_out = nullptr;
   int sms = cfg->num_sms;
@@ -1114,12 +1119,20 @@ int pod_attn_plan(const pod_attn_config* cfg, int32_t prefill_qo_len, int32_t pr
     if (e != cudaSuccess) return cuda_fail(e);
   }
   pod_attn_plan_t* pl = nullptr;
-  const int rc = pod_plan_build(cfg, sms, prefill_qo_len, prefill_kv_len, num_decode, decode_kv_lens, &pl);
+  const int rc = pod_plan_build(cfg, sms, num_prefill, prefill_qo_lens, prefill_kv_lens, num_decode, decode_kv_lens,
+                                &pl);
   if (rc != POD_OK) return rc;
   pl->cfg.num_sms = sms;
   *plan_out = pl;
   if (workspace_bytes_out) *workspace_bytes_out = (size_t)pl->ws_bytes;
   return POD_OK;
+}
+
+int pod_attn_plan(const pod_attn_config* cfg, int32_t prefill_qo_len, int32_t prefill_kv_len,
+                  int32_t num_decode, const int32_t* decode_kv_lens,
+                  pod_attn_plan_t** plan_out, size_t* workspace_bytes_out) {
+  return pod_attn_plan_batched(cfg, 1, &prefill_qo_len, &prefill_kv_len, num_decode, decode_kv_lens, plan_out,
+                               workspace_bytes_out);
 }
 
 int pod_attn_plan_get_info(const pod_attn_plan_t* pl, pod_attn_plan_info* info) {
@@ -1141,6 +1154,14 @@ int pod_attn_plan_get_info(const pod_attn_plan_t* pl, pod_attn_plan_info* info) 
   info->kv_bytes = pl->kv_bytes;
   info->qo_bytes = pl->qo_bytes;
   info->table_bytes = (int64_t)pl->image.size();
+  info->num_prefill_requests = pl->NP;
+  info->num_prefill_rows = pl->P;
+  return POD_OK;
+}
+
+int pod_attn_plan_prefill_requests(const pod_attn_plan_t* pl, int32_t* out) {
+  if (!pl) return POD_ERR_INVALID_ARG;
+  if (out && !pl->preq.empty()) std::memcpy(out, pl->preq.data(), pl->preq.size() * 4);
   return POD_OK;
 }
 
@@ -1225,6 +1246,7 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   prm.pre_items = reinterpret_cast<const int4*>(w + pl->off_pre);
   prm.dec_items = reinterpret_cast<const int4*>(w + pl->off_dec);
   prm.merge_items = reinterpret_cast<const int4*>(w + pl->off_merge);
+  prm.pre_reqs = reinterpret_cast<const int4*>(w + pl->off_preq);
   prm.merge_cnt = reinterpret_cast<int32_t*>(w + pl->off_merge_cnt);
   prm.merge_in_kernel = (pl->cfg.flags & POD_FLAG_MERGE_KERNEL) ? 0 : 1;
   prm.selftest_timeout = (pl->cfg.flags & POD_FLAG_SELFTEST_TIMEOUT) ? 1 : 0;
@@ -1239,8 +1261,7 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.g = pl->g;
-  prm.P = pl->P;
-  prm.C = pl->C;
+  prm.NP = pl->NP;
   prm.B = pl->B;
   prm.ratio_p = pl->ratio_p;
   prm.ratio_d = pl->ratio_d;

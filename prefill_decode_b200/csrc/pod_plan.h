@@ -18,14 +18,17 @@ constexpr int kCostRatio = 248;      // B200 tensor FLOP/s per HBM byte/s (1624.
 
 // Workspace layout (bytes).  Counters first, then one completion counter per
 // merge item (both zeroed every run); the tables follow in the order
-// prefill items | decode items | merge items; then split partials.
+// prefill items | decode items | merge items | prefill requests; then split
+// partials.
 constexpr int64_t kCountersBytes = 4096;
 constexpr int kTicketBase = 0;       // int32 [kMaxSms]
 constexpr int kNextPrefill = 512;    // int32
 constexpr int kNextDecode = 513;     // int32
 constexpr int kErrorWord = 514;      // int32 (first error code recorded)
 constexpr int kErrorInfo = 515;      // int32 (item or block that caused it)
-constexpr int kPrefillItemInts = 4;  // q0, q_head, kv_end, partial
+constexpr int kPrefillItemInts = 4;  // q0 (within the request), q_head, kv_end, prefill request
+constexpr int kPrefillReqInts = 4;   // q_start (row of q_prefill), P, C, 0
+constexpr int kMaxPrefillRequests = 4096;
 constexpr int kDecodeItemInts = 8;   // r, kv_head, k0, k1, partial, merge item, splits, 0
 constexpr int kMergeItemInts = 4;    // r, kv_head, first_partial, num_splits
 
@@ -35,19 +38,21 @@ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct pod_attn_plan {
   pod_attn_config cfg;      // as given, with defaults resolved
-  int32_t P = 0, C = 0, B = 0, g = 1;
+  int32_t NP = 0, P = 0, B = 0, g = 1;   // prefill requests, their query rows in total, decodes
   int32_t n_pre = 0, n_dec = 0, n_merge = 0, n_part = 0;
   int32_t ctas = 2, ratio_p = 1, ratio_d = 1, chunk_pages = 16, num_sms = 148, grid = 0;
   int64_t off_merge_cnt = 0;   // int32 per merge item: splits finished (reset to 0 by the merging warp)
-  int64_t off_pre = 0, off_dec = 0, off_merge = 0, off_part_o = 0, off_part_lse = 0, ws_bytes = 0;
+  int64_t off_pre = 0, off_dec = 0, off_merge = 0, off_preq = 0, off_part_o = 0, off_part_lse = 0, ws_bytes = 0;
   int64_t prefill_flops = 0, decode_flops = 0, kv_bytes = 0, qo_bytes = 0;
   std::vector<int32_t> decode_lens;
-  std::vector<int32_t> pre, dec, merge;     // host tables
+  std::vector<int32_t> pre, dec, merge, preq;   // host tables
   std::vector<uint8_t> image;                // host image of workspace [kCountersBytes, off_part_o)
   void* ev_start = nullptr;
   void* ev_stop = nullptr;
 };
 
 // Implemented in plan.cpp (pure host code, no CUDA calls).
-int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t P, int32_t kv_len_prefill,
-                   int32_t B, const int32_t* lens, pod_attn_plan_t** out);
+// Request rows of the block table and kv_lens: prefill requests 0..NP-1, then
+// decode requests NP..NP+B-1.
+int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const int32_t* prefill_qo_lens,
+                   const int32_t* prefill_kv_lens, int32_t B, const int32_t* lens, pod_attn_plan_t** out);

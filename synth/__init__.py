@@ -14,10 +14,12 @@ Recipe (every config):
   rng = numpy.random.default_rng(seed); draws in this order:
     1. decode lengths (fixed list, integer uniform with inclusive bounds, or
        lognormal: clip(round_half_even(exp(ln(median) + sigma * z)), lo, hi));
-    2. block permutation rng.permutation(num_blocks); request 0 (the prefill
-       request, kv_len = C + P) takes the first pages, then decodes in order;
-       EXTRA_BLOCKS trailing blocks stay unreferenced;
-    3. Q_prefill [P, Hq, d]; 4. Q_decode [B, Hq, d];
+    2. block permutation rng.permutation(num_blocks); the prefill requests
+       (one by default: request 0, kv_len = C + P; a batched workload lists
+       several (P_i, C_i), rows 0..NP-1) take the first pages, then decodes in
+       order; EXTRA_BLOCKS trailing blocks stay unreferenced;
+    3. Q_prefill [sum P_i, Hq, d] (the requests' rows one after another);
+    4. Q_decode [B, Hq, d];
     5. K pool [num_blocks, Hkv, 16, d]; 6. V pool (same shape);
   values are float32 standard normals drawn in chunks of CHUNK elements and
   rounded to bf16 (round to nearest even).  Slots past a request's length in its
@@ -82,6 +84,22 @@ class Workload:
     lens_args: tuple          # fixed: the lengths; uniform: (lo, hi); lognormal: (median, sigma, lo, hi)
     seed: int
     scale: Optional[float] = None   # default 1/sqrt(head_dim)
+    prefill_reqs: Optional[tuple] = None   # ((P_i, C_i), ...): several prefill requests, rows 0..NP-1
+
+    @property
+    def prefill_requests(self) -> List[tuple]:
+        """(P_i, C_i) per prefill request; one request (row 0, P may be 0) unless batched."""
+        if self.prefill_reqs is not None:
+            return [(int(P), int(C)) for P, C in self.prefill_reqs]
+        return [(self.prefill_len, self.prefill_ctx)]
+
+    @property
+    def num_prefill(self) -> int:
+        return len(self.prefill_requests)
+
+    @property
+    def prefill_rows(self) -> int:
+        return sum(P for P, _ in self.prefill_requests)
 
     @property
     def softmax_scale(self) -> float:
@@ -114,12 +132,12 @@ def _draw_lengths(rng: np.random.Generator, w: Workload) -> np.ndarray:
 @dataclasses.dataclass
 class Batch:
     workload: Workload
-    q_prefill: np.ndarray     # uint16 bf16 bits [P, Hq, d]
+    q_prefill: np.ndarray     # uint16 bf16 bits [sum P_i, Hq, d]
     q_decode: np.ndarray      # uint16 bf16 bits [B, Hq, d]
     k_pool: np.ndarray        # uint16 bf16 bits [num_blocks, Hkv, 16, d]
     v_pool: np.ndarray        # uint16 bf16 bits [num_blocks, Hkv, 16, d]
-    block_table: np.ndarray   # int32 [1 + B, max_pages]; row 0 = prefill request
-    kv_lens: np.ndarray       # int32 [1 + B]; [0] = C + P, [1 + r] = L_r
+    block_table: np.ndarray   # int32 [NP + B, max_pages]; rows 0..NP-1 = prefill requests
+    kv_lens: np.ndarray       # int32 [NP + B]; [i] = C_i + P_i, [NP + r] = L_r
     scale: float
 
     @property
@@ -131,8 +149,20 @@ class Batch:
         return self.workload.prefill_ctx
 
     @property
+    def num_prefill(self) -> int:
+        return self.workload.num_prefill
+
+    @property
+    def prefill_qo_lens(self) -> List[int]:
+        return [P for P, _ in self.workload.prefill_requests]
+
+    @property
+    def prefill_kv_lens(self) -> List[int]:
+        return [int(x) for x in self.kv_lens[:self.num_prefill]]
+
+    @property
     def decode_lens(self) -> np.ndarray:
-        return self.kv_lens[1:]
+        return self.kv_lens[self.num_prefill:]
 
     @property
     def num_blocks(self) -> int:
@@ -142,26 +172,28 @@ class Batch:
 @dataclasses.dataclass
 class Layout:
     """Lengths and paged-block layout of a batch (draws 1 and 2 of the recipe)."""
-    kv_lens: np.ndarray       # int32 [1 + B]
-    block_table: np.ndarray   # int32 [1 + B, max_pages]
+    kv_lens: np.ndarray       # int32 [NP + B]
+    block_table: np.ndarray   # int32 [NP + B, max_pages]
     num_blocks: int
     unused_blocks: np.ndarray # blocks no request references (poison)
 
 
 def make_layout(w: Workload, rng: Optional[np.random.Generator] = None) -> Layout:
-    B, P, C = w.num_decode, w.prefill_len, w.prefill_ctx
+    B = w.num_decode
     rng = np.random.default_rng(w.seed) if rng is None else rng
     dec = _draw_lengths(rng, w)
-    kv_lens = np.concatenate([np.asarray([C + P if P > 0 else 0], dtype=np.int32), dec]).astype(np.int32)
+    pre = [C + P if P > 0 else 0 for P, C in w.prefill_requests]
+    kv_lens = np.concatenate([np.asarray(pre, dtype=np.int32), dec]).astype(np.int32)
     pages = (kv_lens.astype(np.int64) + PAGE - 1) // PAGE
     used = int(pages.sum())
     num_blocks = used + EXTRA_BLOCKS
     perm = rng.permutation(num_blocks).astype(np.int32)
     poison_block = int(perm[used])
     max_pages = max(1, int(pages.max()) if pages.size else 1)
-    bt = np.full((1 + B, max_pages), poison_block, dtype=np.int32)
+    R = len(pre) + B
+    bt = np.full((R, max_pages), poison_block, dtype=np.int32)
     off = 0
-    for r in range(1 + B):
+    for r in range(R):
         n = int(pages[r])
         bt[r, :n] = perm[off:off + n]
         off += n
@@ -170,7 +202,7 @@ def make_layout(w: Workload, rng: Optional[np.random.Generator] = None) -> Layou
 
 def make_batch(w: Workload) -> Batch:
     Hq, Hkv, d = w.num_q_heads, w.num_kv_heads, w.head_dim
-    P, C, B = w.prefill_len, w.prefill_ctx, w.num_decode
+    P, B = w.prefill_rows, w.num_decode
     rng = np.random.default_rng(w.seed)
     lay = make_layout(w, rng)
     kv_lens, bt, num_blocks = lay.kv_lens, lay.block_table, lay.num_blocks
@@ -183,7 +215,7 @@ def make_batch(w: Workload) -> Batch:
     v_pool = _normal_bf16(rng, (num_blocks, Hkv, PAGE, d))
     pk = f32_to_bf16_bits(np.float32(POISON_K)).item()
     pv = f32_to_bf16_bits(np.float32(POISON_V)).item()
-    for r in range(1 + B):
+    for r in range(len(kv_lens)):
         L, n = int(kv_lens[r]), int(pages[r])
         if n and L % PAGE:
             blk = bt[r, n - 1]
@@ -241,11 +273,19 @@ def sweep_points() -> List[Workload]:
     return pts
 
 
+def batched_llama3_8b_mix(seed: int = 4) -> Workload:
+    """Batched hybrid batch: three prefill chunks (512 over 3584, 512 over 1536,
+    256 over 0 prior tokens) + 64 decodes U[1024,4096]; 32/8 heads, d=128."""
+    return Workload("batched_llama3_8b_mix", 32, 8, 128, 0, 0, 64, "uniform", (1024, 4096), seed,
+                    prefill_reqs=((512, 3584), (512, 1536), (256, 0)))
+
+
 NAMED = {
     "tiny": tiny,
     "llama3_8b_mix": llama3_8b_mix,
     "long_context_mix": long_context_mix,
     "decode_heavy_mix": decode_heavy_mix,
+    "batched_llama3_8b_mix": batched_llama3_8b_mix,
 }
 
 
@@ -253,3 +293,11 @@ def custom(name: str, Hq: int, Hkv: int, d: int, P: int, C: int, lens: Sequence[
            scale: Optional[float] = None) -> Workload:
     """Small hand-sized batch (fixed decode lengths) for edge-case tests."""
     return Workload(name, Hq, Hkv, d, P, C if P > 0 else 0, len(lens), "fixed", tuple(int(x) for x in lens), seed, scale)
+
+
+def custom_batched(name: str, Hq: int, Hkv: int, d: int, prefill_reqs: Sequence[tuple], lens: Sequence[int],
+                   seed: int, scale: Optional[float] = None) -> Workload:
+    """Small batched hybrid batch: prefill requests ((P_i, C_i), ...) in rows
+    0..NP-1, fixed decode lengths after them."""
+    return Workload(name, Hq, Hkv, d, 0, 0, len(lens), "fixed", tuple(int(x) for x in lens), seed, scale,
+                    prefill_reqs=tuple((int(P), int(C)) for P, C in prefill_reqs))

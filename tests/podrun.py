@@ -21,10 +21,13 @@ class _LayoutBatch:
         self.scale = w.softmax_scale
         self.prefill_len = w.prefill_len
         self.prefill_ctx = w.prefill_ctx
+        self.num_prefill = w.num_prefill
+        self.prefill_qo_lens = [P for P, _ in w.prefill_requests]
+        self.prefill_kv_lens = [int(x) for x in lay.kv_lens[:w.num_prefill]]
 
     @property
     def decode_lens(self):
-        return self.kv_lens[1:]
+        return self.kv_lens[self.num_prefill:]
 
 
 class DeviceBatch:
@@ -37,7 +40,7 @@ class DeviceBatch:
         lay = synth.make_layout(w)
         gen = torch.Generator(device=device)
         gen.manual_seed(w.seed)
-        Hq, Hkv, d, P, B = w.num_q_heads, w.num_kv_heads, w.head_dim, w.prefill_len, w.num_decode
+        Hq, Hkv, d, P, B = w.num_q_heads, w.num_kv_heads, w.head_dim, w.prefill_rows, w.num_decode
 
         def normal(*shape):
             return torch.randn(*shape, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
@@ -68,7 +71,7 @@ class DeviceBatch:
         self.b = b
         w = b.workload
         self.torch = torch
-        self.q_pre = bits_to_bf16(torch, b.q_prefill, device) if w.prefill_len else None
+        self.q_pre = bits_to_bf16(torch, b.q_prefill, device) if w.prefill_rows else None
         self.q_dec = bits_to_bf16(torch, b.q_decode, device) if w.num_decode else None
         self.k = bits_to_bf16(torch, b.k_pool, device)
         self.v = bits_to_bf16(torch, b.v_pool, device)
@@ -79,6 +82,9 @@ class DeviceBatch:
 
     def plan(self, pod, **kw):
         w = self.b.workload
+        if w.prefill_reqs is not None:   # several prefill requests: the batched planner
+            return pod.Plan(w.num_q_heads, w.num_kv_heads, w.head_dim, self.b.prefill_qo_lens,
+                            self.b.prefill_kv_lens, self.b.decode_lens, **kw)
         P, C = w.prefill_len, w.prefill_ctx
         return pod.Plan(w.num_q_heads, w.num_kv_heads, w.head_dim, P, C + P, self.b.decode_lens, **kw)
 

@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 import synth
-from oracle.plan_ref import plan_ref, PlanError
+from oracle.plan_ref import plan_ref, plan_ref_batched, PlanError
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -108,6 +108,57 @@ def test_c_plan_rejects(pod, bad, code):
     with pytest.raises(PlanError):
         plan_ref(a["Hq"], a["Hkv"], a["d"], a["sms"], a["P"], a["KV"], a["lens"], page_size=a["page"],
                  ctas_per_sm=a["ctas"], ratio_p=a["ratio"][0], ratio_d=a["ratio"][1])
+
+
+def _compare_batched(pod, Hq, Hkv, d, sms, qo, kv, lens, **kw):
+    ref = plan_ref_batched(Hq, Hkv, d, sms, qo, kv, lens, **kw)
+    ratio = (kw.get("ratio_p", 0), kw.get("ratio_d", 0))
+    pl = pod.Plan(Hq, Hkv, d, qo, kv, lens, num_sms=sms, ctas_per_sm=kw.get("ctas_per_sm", 0), ratio=ratio,
+                  max_waves=kw.get("max_waves", 0), min_chunk_pages=kw.get("min_chunk_pages", 0))
+    pre, dec, mer = pl.tables()
+    np.testing.assert_array_equal(pre, ref.prefill_items)
+    np.testing.assert_array_equal(dec, ref.decode_items)
+    np.testing.assert_array_equal(mer, ref.merge_items)
+    np.testing.assert_array_equal(pl.prefill_requests(), ref.prefill_requests)
+    i = pl.info
+    assert (i.ctas_per_sm, i.ratio_prefill, i.ratio_decode, i.chunk_pages, i.num_partials) == (
+        ref.ctas_per_sm, ref.ratio_p, ref.ratio_d, ref.chunk_pages, ref.num_partials)
+    assert (i.num_prefill_requests, i.num_prefill_rows) == (len(qo), sum(qo))
+    # algorithmic counts over every prefill request
+    assert i.prefill_flops == 4 * d * Hq * sum(sum(K - P + j + 1 for j in range(P)) for P, K in zip(qo, kv))
+    assert i.kv_bytes == 4 * d * Hkv * (sum(K for P, K in zip(qo, kv) if P > 0) + sum(lens))
+    assert i.qo_bytes == 4 * d * Hq * (sum(qo) + len(lens))
+    return pl
+
+
+def test_c_batched_plan_matches_plan_ref_random(pod):
+    rng = np.random.default_rng(77)
+    for _ in range(60):
+        Hkv = int(rng.choice([1, 2, 8]))
+        g = int(rng.choice([1, 4, 8]))
+        NP = int(rng.integers(0, 7))
+        qo = [int(rng.choice([0, 1, 64, 128, 300, 1025])) for _ in range(NP)]
+        kv = [P + (int(rng.integers(0, 3000)) if P else int(rng.integers(0, 5))) for P in qo]
+        lens = [int(x) for x in rng.integers(1, 6000, size=int(rng.integers(0, 30)))]
+        kw = dict(ctas_per_sm=int(rng.choice([0, 1, 2])), max_waves=int(rng.choice([0, 1, 3])),
+                  min_chunk_pages=int(rng.choice([0, 1, 16])))
+        _compare_batched(pod, Hkv * g, Hkv, int(rng.choice([64, 128])), int(rng.integers(1, 200)), qo, kv, lens, **kw)
+
+
+def test_c_single_form_equals_one_request_batch(pod):
+    a = pod.Plan(32, 8, 128, 512, 4608, [1000, 3000], num_sms=148)
+    b = pod.Plan(32, 8, 128, [512], [4608], [1000, 3000], num_sms=148)
+    for x, y in zip(a.tables(), b.tables()):
+        np.testing.assert_array_equal(x, y)
+    np.testing.assert_array_equal(a.prefill_requests(), b.prefill_requests())
+    assert a.workspace_bytes == b.workspace_bytes
+
+
+@pytest.mark.parametrize("qo,kv", [([-1], [5]), ([10], [5]), ([1 << 24, 1], [1 << 24, 1])])
+def test_c_batched_plan_rejects(pod, qo, kv):
+    with pytest.raises(pod.PodError) as e:
+        pod.Plan(8, 2, 128, qo, kv, [100], num_sms=148)
+    assert e.value.status == pod.POD_ERR_INVALID_ARG
 
 
 def test_run_rejects_bad_host_arguments(pod):

@@ -266,3 +266,75 @@ def test_planted_gqa_mapping_mistake_is_caught(monkeypatch):
             wrong[r, h] = A.attend_rows(q[r, h:h + 1], K, V, b.scale, [L])[0]
     ref = A.attend_decode(b.q_decode, kp_rep, vp_rep, b.block_table, b.kv_lens, b.scale, 8)
     assert np.abs(wrong - ref).max() > 1e-3
+
+
+# ----------------------------------------------- several prefill requests (batched)
+
+def _tiny_batched(seed):
+    w = synth.custom_batched("tiny_batched", 4, 2, 8, [(5, 3), (1, 0), (0, 0), (7, 9)], [6, 17, 1], seed,
+                             scale=0.35)
+    return synth.make_batch(w)
+
+
+@pytest.mark.parametrize("seed", [41, 42])
+def test_batched_oracle_matches_brute_force(seed):
+    """Each prefill request reads its own block-table row and its own prior
+    context; decodes start after the prefill rows (brute-force loops)."""
+    b = _tiny_batched(seed)
+    Hkv = b.workload.num_kv_heads
+    got = A.attend_prefill_batched(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_qo_lens,
+                                   b.prefill_kv_lens, b.scale, Hkv)
+    parts, start = [], 0
+    for i, (P, K) in enumerate(zip(b.prefill_qo_lens, b.prefill_kv_lens)):
+        if P:
+            parts.append(A.attend_brute_prefill(b.q_prefill[start:start + P], b.k_pool, b.v_pool, b.block_table,
+                                                K - P, b.scale, Hkv, bt_row=i))
+        start += P
+    np.testing.assert_allclose(got, np.concatenate(parts), rtol=0, atol=1e-12)
+    gd = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, Hkv,
+                         first_row=b.num_prefill)
+    bd = A.attend_brute_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, Hkv,
+                               first_row=b.num_prefill)
+    np.testing.assert_allclose(gd, bd, rtol=0, atol=1e-12)
+
+
+def test_batched_request_order_invariance():
+    """Reordering the prefill requests (their block-table rows, lengths and Q
+    rows together) reorders the outputs and changes nothing else."""
+    b = _tiny_batched(43)
+    Hkv = b.workload.num_kv_heads
+    qo, kv = b.prefill_qo_lens, b.prefill_kv_lens
+    ref = A.attend_prefill_batched(b.q_prefill, b.k_pool, b.v_pool, b.block_table, qo, kv, b.scale, Hkv)
+    starts = np.concatenate([[0], np.cumsum(qo)])
+    perm = [3, 0, 2, 1]
+    q_perm = np.concatenate([b.q_prefill[starts[i]:starts[i + 1]] for i in perm])
+    bt = b.block_table.copy()
+    bt[:len(qo)] = b.block_table[perm]
+    got = A.attend_prefill_batched(q_perm, b.k_pool, b.v_pool, bt, [qo[i] for i in perm], [kv[i] for i in perm],
+                                   b.scale, Hkv)
+    want = np.concatenate([ref[starts[i]:starts[i + 1]] for i in perm])
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_planted_batched_row_mistake_is_caught(monkeypatch):
+    """A planted mistake -- every prefill request reading block-table row 0 --
+    fails the brute-force pin above."""
+    b = _tiny_batched(44)
+    Hkv = b.workload.num_kv_heads
+    orig = A.attend_prefill
+
+    def always_row0(*args, **kw):
+        kw["bt_row"] = 0
+        return orig(*args, **kw)
+
+    monkeypatch.setattr(A, "attend_prefill", always_row0)
+    got = A.attend_prefill_batched(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_qo_lens,
+                                   b.prefill_kv_lens, b.scale, Hkv)
+    monkeypatch.undo()
+    parts, start = [], 0
+    for i, (P, K) in enumerate(zip(b.prefill_qo_lens, b.prefill_kv_lens)):
+        if P:
+            parts.append(A.attend_brute_prefill(b.q_prefill[start:start + P], b.k_pool, b.v_pool, b.block_table,
+                                                K - P, b.scale, Hkv, bt_row=i))
+        start += P
+    assert np.abs(got - np.concatenate(parts)).max() > 1e-3

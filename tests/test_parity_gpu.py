@@ -37,12 +37,12 @@ def _check(got, ref, what):
 def _oracle(b, pre_rows=None, dec_reqs=None):
     w = b.workload
     op = od = None
-    if w.prefill_len:
-        op = A.attend_prefill(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_ctx, b.scale,
-                              w.num_kv_heads, rows=pre_rows)
+    if w.prefill_rows:
+        op = A.attend_prefill_batched(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_qo_lens,
+                                      b.prefill_kv_lens, b.scale, w.num_kv_heads, rows=pre_rows)
     if w.num_decode:
         od = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale,
-                             w.num_kv_heads, requests=dec_reqs)
+                             w.num_kv_heads, requests=dec_reqs, first_row=b.num_prefill)
     return op, od
 
 
@@ -101,6 +101,42 @@ def test_knobs_keep_results(env, kw):
     rp, rd = _oracle(b)
     _check(op, rp, "prefill")
     _check(od, rd, "decode")
+
+
+BATCHED = [
+    # several prefill requests (rows 0..NP-1): ragged chunks, one row, an empty request, no prior context
+    synth.custom_batched("batched_ragged_d128", 8, 2, 128, [(300, 200), (1, 0), (0, 0), (129, 1000), (64, 64)],
+                         [1, 15, 17, 1000, 3000], 17),
+    synth.custom_batched("batched_d64_g4", 8, 2, 64, [(130, 33), (257, 0)], [700, 64], 18),
+    synth.custom_batched("batched_g7", 28, 4, 128, [(96, 500), (40, 17)], [2100, 5], 20),
+    synth.custom_batched("batched_prefill_only", 32, 8, 128, [(512, 1024), (200, 300), (100, 0)], [], 19),
+]
+
+
+@pytest.mark.parametrize("w", BATCHED, ids=lambda w: w.name)
+@pytest.mark.parametrize("flags", [0, 1, 16], ids=["fused", "sequential", "two_streams"])
+def test_batched_full_parity(env, w, flags):
+    b = synth.make_batch(w)
+    db, pl, ws = _run(env, b, flags=flags)
+    assert pl.info.num_prefill_requests == w.num_prefill
+    op, od = db.outputs()
+    rp, rd = _oracle(b)
+    _check(op, rp, f"{w.name} prefill")
+    if rd is not None:
+        _check(od, rd, f"{w.name} decode")
+
+
+def test_batched_llama3_8b_mix_sampled(env):
+    w = synth.batched_llama3_8b_mix()
+    # first and last rows of each request (rows 0..511, 512..1023, 1024..1279) and a few in between
+    rows = [0, 127, 128, 511, 512, 600, 1023, 1024, 1151, 1279]
+    reqs = [0, 1, 31, 63]
+    b = synth.make_batch(w)
+    db, pl, ws = _run(env, b)
+    op, od = db.outputs()
+    rp, rd = _oracle(b, pre_rows=rows, dec_reqs=reqs)
+    _check(op[rows], rp, "batched prefill rows")
+    _check(od[reqs], rd, "batched decode requests")
 
 
 def _sampled(env, w, pre_rows, dec_reqs, **kw):

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 
 import synth
-from oracle.plan_ref import plan_ref, PlanError, PAGE
+from oracle.plan_ref import plan_ref, plan_ref_batched, PlanError, PAGE
 
 SMS = 148
 
@@ -30,8 +30,8 @@ def check_plan(pl, Hq, Hkv, P, C, lens, sms=SMS, waves=2, minc=16):
     # prefill coverage: each (tile, head) once, kv_end = C + tile end
     T = -(-P // 128)
     seen = set()
-    for q0, h, kv_end, part in pl.prefill_items.tolist():
-        assert q0 % 128 == 0 and 0 <= h < Hq and part == -1
+    for q0, h, kv_end, req in pl.prefill_items.tolist():
+        assert q0 % 128 == 0 and 0 <= h < Hq and req == 0
         assert kv_end == C + min(q0 + 128, P)
         assert (q0, h) not in seen
         seen.add((q0, h))
@@ -148,3 +148,66 @@ def test_plan_rejects(bad):
             args[k] = v
     with pytest.raises(PlanError):
         plan_ref(**args, **kw)
+
+
+def check_prefill_batched(pl, Hq, qo, kv):
+    """Every (request, tile, head) once with its own kv_end, longest first,
+    and a request table of consecutive q_prefill rows."""
+    seen = set()
+    for q0, h, kv_end, req in pl.prefill_items.tolist():
+        P, C = qo[req], kv[req] - qo[req]
+        assert 0 <= req < len(qo) and P > 0
+        assert q0 % 128 == 0 and q0 < P and 0 <= h < Hq
+        assert kv_end == C + min(q0 + 128, P)
+        assert (req, q0, h) not in seen
+        seen.add((req, q0, h))
+    assert len(seen) == sum(-(-P // 128) for P in qo) * Hq
+    ends = pl.prefill_items[:, 2].tolist()
+    assert ends == sorted(ends, reverse=True)
+    start = 0
+    for i, (q_start, P, C, z) in enumerate(pl.prefill_requests.tolist()):
+        assert (q_start, P, z) == (start, qo[i], 0)
+        assert C == (kv[i] - qo[i] if qo[i] > 0 else 0)
+        start += P
+
+
+BATCHED = [
+    ([300, 50, 129], [900, 50, 129], [100, 2000, 17]),
+    ([512, 512, 1024], [4608, 1024, 5120], list(range(300, 6000, 300))),
+    ([0, 200, 0, 7], [10, 300, 0, 7], [64]),
+    ([1536], [1536], []),
+    ([128] * 9, [128 * (i + 1) for i in range(9)], [4096] * 4),
+]
+
+
+@pytest.mark.parametrize("case", BATCHED, ids=lambda c: f"np{len(c[0])}_b{len(c[2])}")
+def test_batched_plan_invariants(case):
+    qo, kv, lens = case
+    pl = plan_ref_batched(8, 2, 128, SMS, qo, kv, lens)
+    check_prefill_batched(pl, 8, qo, kv)
+    # the decode side is planned exactly as with one prefill request of the same work
+    one = plan_ref(8, 2, 128, SMS, 0, 0, lens)
+    assert np.array_equal(pl.decode_items, one.decode_items)
+    assert np.array_equal(pl.merge_items, one.merge_items)
+
+
+def test_batched_one_request_is_the_single_form():
+    a = plan_ref(32, 8, 128, SMS, 512, 4608, [1000, 2500, 4096])
+    b = plan_ref_batched(32, 8, 128, SMS, [512], [4608], [1000, 2500, 4096])
+    for f in ("prefill_items", "decode_items", "merge_items", "prefill_requests"):
+        assert np.array_equal(getattr(a, f), getattr(b, f))
+    assert (a.ratio_p, a.ratio_d, a.chunk_pages) == (b.ratio_p, b.ratio_d, b.chunk_pages)
+
+
+def test_batched_ratio_counts_every_request():
+    # many prefill requests make the batch prefill-heavy; the same work in one request plans the same ratio
+    many = plan_ref_batched(32, 8, 128, SMS, [512] * 8, [4608] * 8, [2048] * 4, ctas_per_sm=1)
+    assert (many.ratio_p, many.ratio_d) == (1, 0)
+    mixed = plan_ref_batched(32, 8, 128, SMS, [512, 512], [4608, 4608], [2048] * 64)
+    assert (mixed.ratio_p, mixed.ratio_d) == (1, 1)
+
+
+@pytest.mark.parametrize("qo,kv", [([-1], [5]), ([10], [5]), ([10, 5], [10]), ([1 << 24, 1], [1 << 24, 1])])
+def test_batched_rejects(qo, kv):
+    with pytest.raises(PlanError):
+        plan_ref_batched(8, 2, 128, SMS, qo, kv, [100])
