@@ -273,9 +273,12 @@ def run_sweep(args):
     for w in wls:
         db = DeviceBatch.generated_on_device(torch, w)
         res = {"workload": w.name, "values": "torch.Generator(cuda, seed) normals; layout from synth"}
-        for mode, flags in (("fused", 0), ("sequential", pod.POD_FLAG_SEQUENTIAL),
-                            ("two_streams", pod.POD_FLAG_TWO_STREAMS)):
-            pl = db.plan(pod, flags=flags)
+        arms = (("fused", {}), ("sequential", dict(flags=pod.POD_FLAG_SEQUENTIAL)),
+                ("two_streams", dict(flags=pod.POD_FLAG_TWO_STREAMS)))
+        if args.sweep_ratios:
+            arms += (("fused_1_1", dict(ratio=(1, 1))), ("fused_1_0", dict(ratio=(1, 0))))
+        for mode, kw in arms:
+            pl = db.plan(pod, **kw)
             ws = db.workspace(pl)
             pl.upload(ws, stream)
             ev = [(pod.Event(), pod.Event()) for _ in range(args.steps)]
@@ -320,6 +323,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--sweep-ratios", action="store_true",
+                    help="sweep mode: also time the fused kernel at forced role ratios 1:1 and 1:0")
     ap.add_argument("--sweep", default=None,
                     help="'all' or comma-separated workload names: per-workload table lines instead of the bench line")
     args = ap.parse_args()

@@ -41,7 +41,11 @@ Rule
     cost_dec = 248 * 4 d Hkv sum_r L_r (bytes x 248, the measured B200
     tensor-FLOP/s per HBM-byte/s); k = ctas_per_sm;
     n_p = floor((2 k cost_pre + tot) / (2 tot)), tot = cost_pre + cost_dec,
-    clamped to [1, k-1] when k >= 2 and n_p = 1 when k = 1; (p, d) = (n_p, k - n_p)
+    clamped to [1, k-1] when k >= 2 and n_p = 1 when k = 1; but n_p = k when
+    2 cost_pre >= tot (the prefill side dominates: every CTA starts prefill-first
+    and decode fills in as CTAs run out of prefill items; measured on B200, this
+    beats 1:1 by ~16% exactly on the sweep points where it applies and loses
+    where decode holds more than half the roofline cost); (p, d) = (n_p, k - n_p)
     reduced by gcd (k = 1 gives 1:0).
 """
 from __future__ import annotations
@@ -191,6 +195,8 @@ def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms
             n_p = min(max(n_p, 1), k - 1)
         else:
             n_p = 1
+        if 2 * cost_pre >= tot:
+            n_p = k
         p_, d_ = n_p, k - n_p
         if d_ == 0:
             p_ = 1

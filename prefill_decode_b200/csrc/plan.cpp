@@ -183,6 +183,7 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
     int64_t n_p = (int64_t)((2 * (__int128)k * cost_pre + tot) / (2 * tot));
     if (k >= 2) n_p = std::min<int64_t>(std::max<int64_t>(n_p, 1), k - 1);
     else n_p = 1;
+    if (2 * cost_pre >= tot) n_p = k;   // prefill dominates: every CTA prefill-first, decode fills in
     rp = (int32_t)n_p;
     rd = k - rp;
     if (rd == 0) {
