@@ -12,7 +12,7 @@ namespace pod {
 constexpr int kPage = 16;            // tokens per KV page
 constexpr int kBM = 128;             // prefill query-tile rows (= TMEM lanes)
 constexpr int kBN = 64;              // prefill key-tile columns
-constexpr int kWarpsPerCta = 4;      // 128-thread CTAs; 4 single-warp decode units
+constexpr int kWarpsPerCta = 4;      // softmax / single-warp decode warps per CTA (plus the MMA and TMA warps)
 constexpr int kMaxSms = 512;         // ticket slots (smid is folded modulo this)
 constexpr int kCostRatio = 248;      // B200 tensor FLOP/s per HBM byte/s (1624.7e12 / 6539.5e9)
 
