@@ -137,3 +137,32 @@ def test_schedule_trace(env, ratio):
     rows = [0, 255, 256, 511]
     assert _close(op[rows], A.attend_prefill(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_ctx,
                                              b.scale, 8, rows=rows))
+
+
+def test_out_of_range_block_id_in_a_batched_prefill_request(env):
+    """A bad block id in prefill request 1 of a batched batch (its own
+    block-table row) is reported in the error word; request 0 and the decodes
+    are untouched."""
+    torch, pod = env
+    w = synth.custom_batched("robust_batched", 8, 2, 128, [(100, 300), (130, 200)], [500, 40], 33)
+    b = synth.make_batch(w)
+    db = DeviceBatch(torch, b)
+    bt = b.block_table.copy()
+    bad = 10 ** 7
+    bt[1, 3] = bad                      # prefill request 1, page 3 (keys 48..63)
+    db.bt = torch.from_numpy(bt).cuda()
+    pl = db.plan(pod)
+    ws = db.workspace(pl)
+    pl.upload(ws)
+    db.run(pod, pl, ws)
+    torch.cuda.synchronize()
+    assert db.error_word(pl, ws) == pod.POD_ERR_BOUNDS
+    off = pl.info.error_offset
+    assert int(ws[off + 4:off + 8].view(torch.int32).item()) == bad
+    op, od = db.outputs()
+    rp = A.attend_prefill_batched(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_qo_lens,
+                                  b.prefill_kv_lens, b.scale, 2, rows=range(100))
+    assert _close(op[:100], rp)
+    rd = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, 2, first_row=2)
+    assert _close(od, rd)
+    assert np.isfinite(op[100:]).all()
