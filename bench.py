@@ -276,7 +276,8 @@ def run_sweep(args):
         arms = (("fused", {}), ("sequential", dict(flags=pod.POD_FLAG_SEQUENTIAL)),
                 ("two_streams", dict(flags=pod.POD_FLAG_TWO_STREAMS)))
         if args.sweep_ratios:
-            arms += (("fused_1_1", dict(ratio=(1, 1))), ("fused_1_0", dict(ratio=(1, 0))))
+            arms += (("fused_1_1", dict(ratio=(1, 1))), ("fused_1_0", dict(ratio=(1, 0))),
+                     ("sm_partition", dict(flags=pod.POD_FLAG_SM_PARTITION)))
         for mode, kw in arms:
             pl = db.plan(pod, **kw)
             ws = db.workspace(pl)
@@ -409,6 +410,7 @@ def main():
     k_abl = max(50, args.steps // 4)
     ablations = {}
     for name, kw in (("two_streams", dict(flags=pod.POD_FLAG_TWO_STREAMS)),
+                     ("sm_partition", dict(flags=pod.POD_FLAG_SM_PARTITION)),
                      ("prefill_first_1_0", dict(ratio=(1, 0))), ("decode_first_0_1", dict(ratio=(0, 1)))):
         pl_a = db.plan(pod, **kw)
         ws_a = db.workspace(pl_a)
@@ -515,6 +517,7 @@ def main():
         "sequential_us": seq_us, "sequential_kernels_us": seq_kern_us, "speedup_vs_sequential": seq_us / us,
         "ablations": dict(ablations, fused_step_us=us,
                           note="two_streams = prefill-only and decode-only kernels on concurrent streams; "
+                               "sm_partition = roles by SM id instead of per-SM tickets; "
                                "x_first = ratio p:d forced so every CTA starts on that role"),
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
         "plan": {"prefill_items": info.num_prefill_items, "decode_items": info.num_decode_items,

@@ -77,6 +77,10 @@ enum {
                                     decode-only kernel on a library-owned stream forked from it and
                                     joined back with events (concurrent kernels, no co-location
                                     control); ignored with POD_FLAG_SEQUENTIAL */
+#define POD_FLAG_SM_PARTITION 32u /* ablation of the per-SM tickets: in the fused kernel every CTA on
+                                     one of the first ceil(prefill items / CTAs per SM) SM ids starts
+                                     prefill-first and every other CTA decode-first (both still steal),
+                                     so prefill and decode mostly run on separate SMs */
 
 typedef struct pod_attn_config {
   int32_t num_q_heads;      /* Hq */

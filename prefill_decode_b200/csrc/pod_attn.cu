@@ -72,6 +72,7 @@ struct alignas(64) PodParams {
   int32_t use_tmem;
   int32_t merge_in_kernel; // 1: the warp finishing a row's last split merges the row
   int32_t selftest_timeout; // 1: CTA 0 exercises the expired-wait path once
+  int32_t partition_sms;   // > 0: roles by SM id instead of per-SM tickets (ablation)
   float scale_log2;        // softmax scale * log2(e)
 };
 
@@ -856,7 +857,10 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
     tma_prefetch_desc(&p.tm_kp);
     tma_prefetch_desc(&p.tm_vp);
     int home = p.mode == kDecodeOnly ? kRoleDecode : kRolePrefill;
-    if (p.mode == kFused) {
+    if (p.mode == kFused && p.partition_sms > 0) {
+      // ablation: whole SMs start on one role (the first partition_sms SM ids prefill-first)
+      home = (int)smid() < p.partition_sms ? kRolePrefill : kRoleDecode;
+    } else if (p.mode == kFused) {
       const uint32_t sm = smid();
       const int t = atomicAdd(&p.counters[kTicketBase + (int)(sm % kMaxSms)], 1);
       const int span = p.ratio_p + p.ratio_d;
@@ -1250,6 +1254,11 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   prm.merge_cnt = reinterpret_cast<int32_t*>(w + pl->off_merge_cnt);
   prm.merge_in_kernel = (pl->cfg.flags & POD_FLAG_MERGE_KERNEL) ? 0 : 1;
   prm.selftest_timeout = (pl->cfg.flags & POD_FLAG_SELFTEST_TIMEOUT) ? 1 : 0;
+  if ((pl->cfg.flags & POD_FLAG_SM_PARTITION) && pl->n_pre > 0 && pl->n_dec > 0) {
+    // as many SMs as the prefill items fill with every CTA of the SM, at least one, at most all
+    const int64_t want = ((int64_t)pl->n_pre + pl->ctas - 1) / pl->ctas;
+    prm.partition_sms = (int32_t)(want < 1 ? 1 : (want > pl->num_sms ? pl->num_sms : want));
+  }
   prm.part_o = reinterpret_cast<float*>(w + pl->off_part_o);
   prm.part_lse = reinterpret_cast<float*>(w + pl->off_part_lse);
   prm.trace = (pl->cfg.flags & POD_FLAG_TRACE) ? trace : nullptr;

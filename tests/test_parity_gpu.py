@@ -90,9 +90,11 @@ def test_small_batches_full_parity(env, w, flags):
 
 @pytest.mark.parametrize("kw", [dict(ctas_per_sm=1), dict(ratio=(0, 1)), dict(ratio=(1, 0)), dict(max_waves=8),
                                 dict(min_chunk_pages=1), dict(num_sms=7), dict(flags=4, max_waves=8),
-                                dict(flags=5, max_waves=8), dict(flags=16), dict(flags=16 | 4, max_waves=8)],
+                                dict(flags=5, max_waves=8), dict(flags=16), dict(flags=16 | 4, max_waves=8),
+                                dict(flags=32)],
                          ids=["one_cta", "decode_first", "prefill_first", "many_splits", "tiny_splits", "few_sms",
-                              "merge_kernel", "merge_kernel_sequential", "two_streams", "two_streams_merge_kernel"])
+                              "merge_kernel", "merge_kernel_sequential", "two_streams", "two_streams_merge_kernel",
+                              "sm_partition"])
 def test_knobs_keep_results(env, kw):
     w = synth.custom("knobs", 8, 2, 128, 300, 700, [16, 33, 1000, 2500, 4096], 12)
     b = synth.make_batch(w)
