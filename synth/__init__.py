@@ -7,8 +7,9 @@ take their inputs from it without sharing any of the method's code.
 
 Workload shapes follow the POD-Attention explainer ("The evaluation": Llama-3-8B
 shapes, contexts 4K-20K, prefill chunks 512-2K) and the paged KV-cache layout of
-the disaggregation blog post ("KV cache size" formula: 2 x layers x kv_heads x
-head_size x bytes per token).
+the blog post "Prefill vs. Decode GPU Utilization Imbalance" (section "How the
+KV cache turns the memory-bandwidth constraint into a capacity crisis": a
+token's cache entry is K and V for every layer and kv head).
 
 Recipe (every config):
   rng = numpy.random.default_rng(seed); draws in this order:
