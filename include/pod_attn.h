@@ -10,8 +10,9 @@
  * Inference" (explainer page, "How POD-Attention overlaps prefill and decode":
  * fuse into one kernel, self-assign roles per SM, 2 threadblocks per SM,
  * single-warp virtual decode blocks, capped KV splits, proportional allocation).
- * Split-KV partial results are combined by a log-sum-exp merge kernel (PAT
- * record: "the final merge performs online softmax").
+ * Split-KV partial results are combined by a log-sum-exp merge (the PAT
+ * catalogue record merges its per-split results with online softmax), done by
+ * the warp that finishes a row's last split.
  *
  * Math (per query head h, kv head h / (Hq/Hkv), natural-base softmax):
  *   prefill row i (absolute position C+i): O = softmax(scale q K[0..C+i]^T) V[0..C+i]

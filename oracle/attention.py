@@ -18,8 +18,8 @@ Readings where the pages are silent (the plainest one in each case):
 
 Split-KV (POD-Attention explainer, "Cap prefill splitting to avoid contention",
 FlashDecoding-style) computes a partial result per key range; the ranges are
-combined by a log-sum-exp merge (PAT record: "the final merge performs online
-softmax").  ``attend_partial`` / ``lse_merge`` state that merge.
+combined by a log-sum-exp merge (the PAT catalogue record merges its per-split
+results with online softmax).  ``attend_partial`` / ``lse_merge`` state that merge.
 """
 from __future__ import annotations
 
