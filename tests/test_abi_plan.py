@@ -179,3 +179,27 @@ def test_run_rejects_bad_host_arguments(pod):
     # upload: too small / misaligned
     assert L.pod_attn_upload(pl.handle, 0x1000, 256, None) == -3
     assert L.pod_attn_upload(pl.handle, 0x1010, ws, None) == -1
+
+
+def test_batched_run_rejects_bad_host_arguments(pod):
+    """A batched plan validates its arguments on the host before any launch."""
+    pl = pod.Plan(4, 2, 64, [64, 0, 30], [192, 0, 40], [64, 100], num_sms=4)
+    ws = pl.workspace_bytes
+    L = pod.lib()
+    assert (pl.info.num_prefill_requests, pl.info.num_prefill_rows) == (3, 94)
+    # prefill rows exist: q_prefill / o_prefill are required and 16-byte aligned
+    assert L.pod_attn_run(pl.handle, None, 16, 16, 16, 10, 16, 4, None, 0.125, 16, 16, 0x1000, ws, None, None) == -1
+    assert L.pod_attn_run(pl.handle, 16, 16, 16, 16, 10, 16, 4, None, 0.125, 24, 16, 0x1000, ws, None, None) == -1
+    # tracing without a trace buffer
+    tr = pod.Plan(4, 2, 64, [64], [192], [64], num_sms=4, flags=pod.POD_FLAG_TRACE)
+    assert L.pod_attn_run(tr.handle, 16, 16, 16, 16, 10, 16, 4, None, 0.125, 16, 16, 0x1000, tr.workspace_bytes,
+                          None, None) == -1
+
+
+def test_decode_only_batched_plan_needs_no_prefill_pointers(pod):
+    pl = pod.Plan(8, 2, 128, [], [], [1, 16, 3000], num_sms=148)
+    assert (pl.info.num_prefill_requests, pl.info.num_prefill_items) == (0, 0)
+    assert pl.prefill_requests().shape == (0, 4)
+    # the workspace holds no prefill table and the decode side is planned as usual
+    one = pod.Plan(8, 2, 128, 0, 0, [1, 16, 3000], num_sms=148)
+    np.testing.assert_array_equal(pl.tables()[1], one.tables()[1])
