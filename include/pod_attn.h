@@ -84,7 +84,7 @@ enum {
                                      so prefill and decode mostly run on separate SMs */
 
 typedef struct pod_attn_config {
-  int32_t num_q_heads;      /* Hq */
+  int32_t num_q_heads;      /* Hq, 1..4096 */
   int32_t num_kv_heads;     /* Hkv; Hq % Hkv == 0 and Hq / Hkv <= 8 */
   int32_t head_dim;         /* d in {64, 128} */
   int32_t page_size;        /* tokens per KV page; must be 16 */
@@ -126,12 +126,13 @@ typedef struct pod_attn_plan_info {
  * (ignored if P == 0); it owns block-table / kv_lens row 0 even when P == 0,
  * and decode request r owns row 1 + r.  decode_kv_lens = host array of B
  * lengths, each >= 1.  The work items, the split-KV partition and the ticket
- * ratio follow the rule documented in oracle/plan_ref.py (the pages fix no
+ * ratio follow the rule documented in oracle/plan_ref.py (the sources fix no
  * formula).  On success *plan_out owns a new plan and *workspace_bytes_out
  * (nullable) receives the device workspace size that pod_attn_upload /
  * pod_attn_run need.  Same as pod_attn_plan_batched with one prefill request.
- * Errors: POD_ERR_INVALID_ARG, POD_ERR_UNSUPPORTED, POD_ERR_CUDA (num_sms == 0
- * and no device could be queried). */
+ * Errors: POD_ERR_INVALID_ARG (also when a work count of pod_attn_plan_info
+ * would not fit int64), POD_ERR_UNSUPPORTED, POD_ERR_CUDA (num_sms == 0 and no
+ * device could be queried). */
 int pod_attn_plan(const pod_attn_config* cfg, int32_t prefill_qo_len, int32_t prefill_kv_len,
                   int32_t num_decode, const int32_t* decode_kv_lens,
                   pod_attn_plan_t** plan_out, size_t* workspace_bytes_out);

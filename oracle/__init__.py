@@ -16,8 +16,8 @@ Contents
 Parity status
   attention.*   pinned by brute force, closed forms and invariants
                 (tests/test_oracle.py, tests/golden/).
-  plan_ref.*    parity unpinned by the pages: the pages fix no split or ratio
-                formula, so the rule is this build's own; it is pinned only by
+  plan_ref.*    parity unpinned by the sources: they fix no split or ratio
+                formula, so the rule is the library's own; it is pinned only by
                 invariants (every (row, key) covered once, caps respected,
                 degenerate batches) and by bit-exact agreement with the C
                 planner, which is a separate implementation of the same rule.

@@ -6,7 +6,7 @@ of all earlier tokens, which live in the KV cache.  Prefill processes a chunk of
 prompt tokens at once (hybrid batching = chunked prefill, "What people did");
 decode processes one new token per request and reads that request's whole cache.
 
-Readings where the pages are silent (the plainest one in each case):
+Readings where the cited sources are silent (the plainest one in each case):
   * weights are softmax(scale * q . k) in the natural base;
   * causal alignment is bottom-right: chunk row i sits at absolute position C+i
     and sees keys 0..C+i (the chunk continues a prompt of C earlier tokens whose

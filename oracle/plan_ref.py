@@ -6,14 +6,16 @@ split-KV capped at two full waves, CTAs allocated in proportion to the batch's
 prefill:decode mix; FlashInfer POD PR "Limit kv split when prefill tokens <=
 1536": the split count accounts for co-located decode CTAs).  This module is
 the written rule that the C planner must reproduce bit for bit.  Parity of the
-plan is therefore unpinned by the pages; tests pin it by invariants.
+plan is therefore unpinned by the sources; tests pin it by invariants.
 
 Rule
-  Validation: Hq % Hkv == 0; g = Hq/Hkv in 1..8; d in {64, 128}; page == 16;
+  Validation: Hq % Hkv == 0, Hq <= 4096; g = Hq/Hkv in 1..8; d in {64, 128}; page == 16;
     1 <= num_sms <= 512; ctas_per_sm in {0 (auto = 2), 1, 2}; ratios >= 0;
     max_waves >= 0 (0 = 2); min_chunk_pages >= 0 (0 = 16); P >= 0;
     if P > 0: P <= prefill_kv_len <= 2^24; 0 <= B <= 65536; 1 <= L_r <= 2^24;
-    sum_r L_r <= 2^31 - 1.
+    sum_r L_r <= 2^31 - 1; every work count reported (4 d Hq sum of keys seen
+    over prefill rows, 4 d Hq sum L_r, 4 d Hkv K/V tokens, 4 d Hq Q/O rows)
+    fits int64.
   Prefill requests i = 0 .. NP-1 (chunk P_i over C_i = kv_i - P_i earlier
     tokens; the one-prefill form is NP = 1, P_0 = P).  Prefill items (one
     128-row query tile of one query head each): for i, for t = T_i-1 .. 0
@@ -62,6 +64,8 @@ WARPS_PER_CTA = 4
 COST_RATIO = 248
 MAX_SMS = 512
 MAX_PREFILL_REQUESTS = 4096
+MAX_HEADS = 4096
+INT64_MAX = (1 << 63) - 1
 
 
 class PlanError(ValueError):
@@ -102,7 +106,7 @@ def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms
     pre_kv = [int(x) for x in prefill_kv_lens]
     lens = [int(x) for x in decode_lens]
     B = len(lens)
-    if Hq <= 0 or Hkv <= 0 or Hq % Hkv:
+    if Hq <= 0 or Hkv <= 0 or Hq % Hkv or Hq > MAX_HEADS:
         raise PlanError("invalid head counts")
     g = Hq // Hkv
     if g > 8 or d not in (64, 128) or page_size != PAGE:
@@ -124,6 +128,12 @@ def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms
     waves = 2 if max_waves == 0 else max_waves
     minc = 16 if min_chunk_pages == 0 else min_chunk_pages
     ctx = [KVp - P if P > 0 else 0 for P, KVp in zip(pre_qo, pre_kv)]
+    # the work counts a plan reports (prefill FLOPs, decode FLOPs, K/V bytes, Q/O bytes) must fit int64
+    rows_keys = sum(P * (C + 1) + P * (P - 1) // 2 for P, C in zip(pre_qo, ctx))
+    pre_kv_tokens = sum(C + P for P, C in zip(pre_qo, ctx) if P > 0)
+    if max(4 * d * Hq * rows_keys, 4 * d * Hq * sum(lens), 4 * d * Hkv * (pre_kv_tokens + sum(lens)),
+           4 * d * Hq * (sum(pre_qo) + B)) > INT64_MAX:
+        raise PlanError("work counts overflow")
 
     # prefill items per request, last tile first; then all requests' items longest first
     pre = []

@@ -18,6 +18,8 @@ namespace {
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+constexpr int kMaxHeads = 4096;   // query heads per plan
+
 struct DecEntry {
   int32_t pages, r, kvh, s;
   int32_t item[pod::kDecodeItemInts];
@@ -30,7 +32,7 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
   using namespace pod;
   if (!cfg || !out) return POD_ERR_INVALID_ARG;
   const int32_t Hq = cfg->num_q_heads, Hkv = cfg->num_kv_heads, d = cfg->head_dim;
-  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return POD_ERR_INVALID_ARG;
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv || Hq > kMaxHeads) return POD_ERR_INVALID_ARG;
   const int32_t g = Hq / Hkv;
   if (g > 8 || (d != 64 && d != 128) || cfg->page_size != kPage) return POD_ERR_UNSUPPORTED;
   if (num_sms < 1 || num_sms > kMaxSms) return POD_ERR_INVALID_ARG;
@@ -52,6 +54,24 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
     sumL += lens[r];
   }
   if (sumL > INT32_MAX) return POD_ERR_INVALID_ARG;
+
+  // ---- algorithmic work (roofline numerators); checked before anything is built
+  int64_t rows_keys = 0, pre_kv_tokens = 0;
+  for (int32_t i = 0; i < NP; ++i) {
+    const int64_t P = pre_qo[i], C = P > 0 ? pre_kv[i] - P : 0;
+    for (int64_t q0 = 0; q0 < P; q0 += kBM) {
+      const int64_t n = std::min<int64_t>(kBM, P - q0);
+      rows_keys += n * (C + 1) + n * q0 + n * (n - 1) / 2;
+    }
+    if (P > 0) pre_kv_tokens += C + P;
+  }
+  {
+    // the work counts must fit the int64 fields they are reported in
+    const __int128 lim = (__int128)INT64_MAX;
+    const __int128 pf = (__int128)4 * d * Hq * rows_keys, df = (__int128)4 * d * Hq * sumL;
+    const __int128 kb = (__int128)4 * d * Hkv * (pre_kv_tokens + sumL), qb = (__int128)4 * d * Hq * (sumP + B);
+    if (pf > lim || df > lim || kb > lim || qb > lim) return POD_ERR_INVALID_ARG;
+  }
 
   pod_attn_plan_t* pl = new (std::nothrow) pod_attn_plan_t();
   if (!pl) return POD_ERR_INVALID_ARG;
@@ -145,16 +165,6 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
   pl->n_merge = (int32_t)(pl->merge.size() / kMergeItemInts);
   pl->n_part = npart;
 
-  // ---- algorithmic work (roofline numerators)
-  int64_t rows_keys = 0, pre_kv_tokens = 0;
-  for (int32_t i = 0; i < NP; ++i) {
-    const int64_t P = pre_qo[i], C = ctx[i];
-    for (int64_t q0 = 0; q0 < P; q0 += kBM) {
-      const int64_t n = std::min<int64_t>(kBM, P - q0);
-      rows_keys += n * (C + 1) + n * q0 + n * (n - 1) / 2;
-    }
-    if (P > 0) pre_kv_tokens += C + P;
-  }
   pl->prefill_flops = 4LL * d * Hq * rows_keys;
   pl->decode_flops = 4LL * d * Hq * sumL;
   pl->kv_bytes = 4LL * d * Hkv * (pre_kv_tokens + sumL);

@@ -203,3 +203,15 @@ def test_decode_only_batched_plan_needs_no_prefill_pointers(pod):
     # the workspace holds no prefill table and the decode side is planned as usual
     one = pod.Plan(8, 2, 128, 0, 0, [1, 16, 3000], num_sms=148)
     np.testing.assert_array_equal(pl.tables()[1], one.tables()[1])
+
+
+def test_c_plan_rejects_too_many_heads_and_overflowing_work(pod):
+    with pytest.raises(pod.PodError) as e:
+        pod.Plan(4104, 513, 128, 64, 128, [100], num_sms=148)
+    assert e.value.status == pod.POD_ERR_INVALID_ARG
+    big = 1 << 24
+    with pytest.raises(pod.PodError) as e:
+        pod.Plan(4096, 512, 128, [big], [big], [100], num_sms=148)
+    assert e.value.status == pod.POD_ERR_INVALID_ARG
+    # the largest head count still plans, and agrees with the planner of record
+    _compare_batched(pod, 4096, 512, 128, 148, [128], [1 << 20], [100])

@@ -211,3 +211,14 @@ def test_batched_ratio_counts_every_request():
 def test_batched_rejects(qo, kv):
     with pytest.raises(PlanError):
         plan_ref_batched(8, 2, 128, SMS, qo, kv, [100])
+
+
+def test_plan_rejects_too_many_heads_and_overflowing_work():
+    """More than 4096 query heads, or work counts past int64, are rejected before anything is built."""
+    with pytest.raises(PlanError):
+        plan_ref(4104, 513, 128, SMS, 64, 128, [100])
+    big = 1 << 24   # 4 d Hq * (about P^2 / 2) keys seen = 2^21 * 2^47 > 2^63
+    with pytest.raises(PlanError):
+        plan_ref_batched(4096, 512, 128, SMS, [big], [big], [100])
+    pl = plan_ref_batched(4096, 512, 128, SMS, [128], [1 << 20], [100])
+    assert len(pl.prefill_items) == 4096 and (pl.prefill_items[:, 2] == 1 << 20).all()
