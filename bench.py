@@ -277,7 +277,8 @@ def run_sweep(args):
                 ("two_streams", dict(flags=pod.POD_FLAG_TWO_STREAMS)))
         if args.sweep_ratios:
             arms += (("fused_1_1", dict(ratio=(1, 1))), ("fused_1_0", dict(ratio=(1, 0))),
-                     ("sm_partition", dict(flags=pod.POD_FLAG_SM_PARTITION)))
+                     ("sm_partition", dict(flags=pod.POD_FLAG_SM_PARTITION)),
+                     ("four_decode_warps", dict(flags=pod.POD_FLAG_DECODE_FOUR_WARPS)))
         for mode, kw in arms:
             pl = db.plan(pod, **kw)
             ws = db.workspace(pl)
@@ -406,17 +407,22 @@ def main():
     clocks = sampler.summary(tw0, tw1)
     seq_ms, seq_kern, _ = timed_loop(seq, ws_seq, max(50, args.steps // 4), True)
     # ablations through the same API: the two kernels of the sequential path on two concurrent streams,
-    # and every CTA starting on one role (the proportional rule gives 1:1 with two CTAs per SM)
+    # roles by SM id, four decode warps per CTA, and every CTA starting on one role (the proportional
+    # rule gives 1:1 with two CTAs per SM)
     k_abl = max(50, args.steps // 4)
     ablations = {}
     for name, kw in (("two_streams", dict(flags=pod.POD_FLAG_TWO_STREAMS)),
                      ("sm_partition", dict(flags=pod.POD_FLAG_SM_PARTITION)),
+                     ("decode_four_warps", dict(flags=pod.POD_FLAG_DECODE_FOUR_WARPS)),
                      ("prefill_first_1_0", dict(ratio=(1, 0))), ("decode_first_0_1", dict(ratio=(0, 1)))):
         pl_a = db.plan(pod, **kw)
         ws_a = db.workspace(pl_a)
         pl_a.upload(ws_a, stream)
-        a_ms, _, _ = timed_loop(pl_a, ws_a, k_abl, False)
-        ablations[name] = {"step_us": max_over_ranks(a_ms * 1e3 / k_abl), "error_word": db.error_word(pl_a, ws_a)}
+        # timed exactly like the fused arm (the same per-step events), so the step times compare directly
+        a_ms, a_kern, _ = timed_loop(pl_a, ws_a, k_abl, True)
+        ablations[name] = {"step_us": max_over_ranks(a_ms * 1e3 / k_abl),
+                           "kernels_us": max_over_ranks(float(np.mean(a_kern)) * 1e3),
+                           "error_word": db.error_word(pl_a, ws_a)}
         del ws_a
     sampler.stop()
     err_word = db.error_word(fused, ws)
@@ -518,6 +524,7 @@ def main():
         "ablations": dict(ablations, fused_step_us=us,
                           note="two_streams = prefill-only and decode-only kernels on concurrent streams; "
                                "sm_partition = roles by SM id instead of per-SM tickets; "
+                               "decode_four_warps = only 4 of a decoding CTA's 6 warps run decode items (deeper page rings); "
                                "x_first = ratio p:d forced so every CTA starts on that role"),
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
         "plan": {"prefill_items": info.num_prefill_items, "decode_items": info.num_decode_items,

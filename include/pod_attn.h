@@ -82,6 +82,10 @@ enum {
                                      one of the first ceil(prefill items / CTAs per SM) SM ids starts
                                      prefill-first and every other CTA decode-first (both still steal),
                                      so prefill and decode mostly run on separate SMs */
+#define POD_FLAG_DECODE_FOUR_WARPS 64u /* ablation: only warps 0-3 of a decoding CTA run decode items
+                                          (page rings 3 deep for d = 128, 4 for d = 64) and the plan's
+                                          split cap counts 4 decode warps per CTA; by default all 6 warps
+                                          decode (the MMA and TMA warps too; rings 2 / 3 deep) */
 
 typedef struct pod_attn_config {
   int32_t num_q_heads;      /* Hq, 1..4096 */

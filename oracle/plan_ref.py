@@ -23,7 +23,8 @@ Rule
     kv_end = C_i + min(128 (t+1), P_i), request i); then stably sorted by
     kv_end, longest first.  Prefill request table (q_start_i = P_0 + .. +
     P_{i-1}, P_i, C_i, 0).
-  Decode split: W = num_sms * ctas_per_sm * 4 decode warps; cap = max_waves * W;
+  Decode split: W = num_sms * ctas_per_sm * decode warps per CTA (6, or 4 in
+    the four-warp ablation); cap = max_waves * W;
     pages_r = ceil(L_r / 16); N = Hkv * sum pages_r; maxp = max pages_r;
     c = max(min_chunk_pages, ceil(N / cap)); then c += 1 while c < maxp and
     Hkv * sum ceil(pages_r / c) > cap.  Decode request r (block-table row
@@ -60,7 +61,7 @@ import numpy as np
 
 PAGE = 16
 BM = 128
-WARPS_PER_CTA = 4
+DECODE_WARPS = 6            # per CTA: every warp decodes (4 in the four-warp ablation)
 COST_RATIO = 248
 MAX_SMS = 512
 MAX_PREFILL_REQUESTS = 4096
@@ -99,7 +100,7 @@ def plan_ref(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
 def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
                      prefill_qo_lens: Sequence[int], prefill_kv_lens: Sequence[int], decode_lens: Sequence[int], *,
                      page_size: int = 16, ctas_per_sm: int = 0, ratio_p: int = 0, ratio_d: int = 0,
-                     max_waves: int = 0, min_chunk_pages: int = 0) -> PlanRef:
+                     max_waves: int = 0, min_chunk_pages: int = 0, decode_warps: int = DECODE_WARPS) -> PlanRef:
     """NP prefill requests (block-table rows 0..NP-1) and B decodes (rows NP..NP+B-1)."""
     Hq, Hkv, d = int(num_q_heads), int(num_kv_heads), int(head_dim)
     pre_qo = [int(x) for x in prefill_qo_lens]
@@ -148,7 +149,9 @@ def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms
         q_start += P
 
     # decode split
-    W = num_sms * k * WARPS_PER_CTA
+    if decode_warps not in (4, 6):
+        raise PlanError("decode warps per CTA must be 4 or 6")
+    W = num_sms * k * decode_warps
     cap = waves * W
     pages = [_ceil(L, PAGE) for L in lens]
     N = Hkv * sum(pages)

@@ -31,6 +31,7 @@ POD_FLAG_MERGE_KERNEL = 4
 POD_FLAG_SELFTEST_TIMEOUT = 8
 POD_FLAG_TWO_STREAMS = 16
 POD_FLAG_SM_PARTITION = 32
+POD_FLAG_DECODE_FOUR_WARPS = 64
 
 EXPORTED = [
     "pod_attn_plan", "pod_attn_plan_get_info", "pod_attn_plan_tables", "pod_attn_upload", "pod_attn_run",

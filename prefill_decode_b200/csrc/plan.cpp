@@ -19,6 +19,7 @@ namespace {
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 constexpr int kMaxHeads = 4096;   // query heads per plan
+constexpr int kDecodeWarpsAll = 6;  // decode warps per CTA when every warp decodes (the kernel's 192 threads)
 
 struct DecEntry {
   int32_t pages, r, kvh, s;
@@ -113,7 +114,9 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
   }
 
   // ---- decode split: chunk c pages, at most waves x decode warps items
-  const int64_t W = (int64_t)num_sms * k * kWarpsPerCta;
+  // decode warps: every warp of the CTA, or warps 0-3 with POD_FLAG_DECODE_FOUR_WARPS
+  const int32_t dwarps = (cfg->flags & POD_FLAG_DECODE_FOUR_WARPS) ? kWarpsPerCta : kDecodeWarpsAll;
+  const int64_t W = (int64_t)num_sms * k * dwarps;
   const int64_t cap = (int64_t)waves * W;
   std::vector<int32_t> pages(B);
   int64_t N = 0;

@@ -73,12 +73,15 @@ struct alignas(64) PodParams {
   int32_t merge_in_kernel; // 1: the warp finishing a row's last split merges the row
   int32_t selftest_timeout; // 1: CTA 0 exercises the expired-wait path once
   int32_t partition_sms;   // > 0: roles by SM id instead of per-SM tickets (ablation)
+  int32_t decode_warps;    // warps of a CTA that run decode items: 4, or 6 (the MMA and TMA warps too)
   float scale_log2;        // softmax scale * log2(e)
 };
 
 constexpr int kThreads = 192;        // warps 0-3: softmax (prefill) / decode units; warp 4: MMA; warp 5: TMA
+                                     // (in decode, warps 4 and 5 idle, or decode too when decode_warps == 6)
 constexpr int kMmaWarp = 4;
 constexpr int kTmaWarp = 5;
+constexpr int kAllWarps = kThreads / 32;
 
 // mbarrier slots in the CTA control block
 enum : int {
@@ -92,7 +95,7 @@ enum : int {
   kBarODone = 13,   // [2] P.V MMA of tile t finished: P buffer and V slot t&1  count 1
                     //     are free again (commit)
   kBarOFinal = 15,  // last P.V MMA of an item finished (commit)                count 1
-  kBarDecode = 16,  // [kWarpsPerCta * kNS] decode page rings                   count 1 + tx
+  kBarDecode = 16,  // [decode warps * ring depth] decode page rings            count 1 + tx
 };
 // Parity waits are only sound when the waiter knows the barrier is at most one
 // phase away from the one it waits for.  For key tile t (counted over the
@@ -119,14 +122,20 @@ struct Cfg {
   static constexpr int kPageBytes = kPage * D * 2;            // one 16-token page of one kv head
   static constexpr int kDecStage = 2 * kPageBytes;            // K page + V page
   static constexpr int kNS = (kPrefillSmem / kWarpsPerCta) / kDecStage;   // decode ring depth per warp
+  static constexpr int kNSAll = (kPrefillSmem / kAllWarps) / kDecStage;    // ... when all warps decode
   static constexpr int kSmem = kPrefillSmem;
-  static constexpr int kNumBars = kBarDecode + kWarpsPerCta * kNS;
+  static constexpr int kNumBars =
+      kBarDecode + (kWarpsPerCta * kNS > kAllWarps * kNSAll ? kWarpsPerCta * kNS : kAllWarps * kNSAll);
   static constexpr int kCtrlBytes = 512;                      // barriers, TMEM address, broadcast slots
   static_assert((kNumBars + 1) * 8 + 32 <= kCtrlBytes, "control block too small");   // + the self-test barrier
   // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) can share an SM
   static constexpr int kSmemAlloc = (kSmem + kCtrlBytes) > 80 * 1024 ? (kSmem + kCtrlBytes) : 80 * 1024;
 };
 static_assert(Cfg<128>::kNS >= 3 && Cfg<64>::kNS >= 3, "decode ring too shallow");
+static_assert(Cfg<128>::kNSAll >= 2 && Cfg<64>::kNSAll >= 2, "decode ring too shallow");
+static_assert(kAllWarps * Cfg<128>::kNSAll * Cfg<128>::kDecStage <= Cfg<128>::kPrefillSmem &&
+                  kAllWarps * Cfg<64>::kNSAll * Cfg<64>::kDecStage <= Cfg<64>::kPrefillSmem,
+              "decode rings exceed the shared-memory union");
 
 __device__ __forceinline__ void record_error(const PodParams& p, int code, int info) {
   if (atomicCAS(&p.counters[kErrorWord], 0, code) == 0) atomicExch(&p.counters[kErrorInfo], info);
@@ -494,11 +503,11 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
 // O^T[d x 8] += V_page^T . P^T.  Pages arrive by TMA into a kNS-deep ring.
 // The block ids of an item's pages are read 32 at a time, one per lane, a
 // window ahead of use, so refilling a ring slot never waits on a global load.
-template <int D>
+template <int D, int NS>
 __device__ __forceinline__ void decode_issue_page(const PodParams& p, uint8_t* ring, uint64_t* wbars, uint32_t seq,
                                                   int blk, int kvh) {
   using CF = Cfg<D>;
-  const int s = seq % CF::kNS;
+  const int s = seq % NS;
   uint8_t* kbuf = ring + s * CF::kDecStage;
   uint64_t* bar = &wbars[s];
   mbar_arrive_expect_tx(bar, CF::kDecStage);
@@ -615,7 +624,7 @@ __device__ void merge_row_warp(const PodParams& p, int midx) {
   }
 }
 
-template <int D>
+template <int D, int NS>
 __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, uint32_t& seq,
                             volatile int* abort_flag, int home_role) {
   using CF = Cfg<D>;
@@ -640,10 +649,10 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
     const int len_now = (lane == 0 && p.kv_lens) ? __ldg(&p.kv_lens[p.NP + r]) : k1;
     int win = 0;
     {
-      const int pre = np < CF::kNS ? np : CF::kNS;
+      const int pre = np < NS ? np : NS;
       for (int j = 0; j < pre; ++j) {
         const int blk = __shfl_sync(0xffffffffu, bt_cur, j);
-        if (lane == 0) decode_issue_page<D>(p, ring, wbars, seq + j, blk, kvh);
+        if (lane == 0) decode_issue_page<D, NS>(p, ring, wbars, seq + j, blk, kvh);
       }
     }
     if (lane == 0) {
@@ -685,8 +694,8 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
     int jfail = 0;
     for (int j = 0; j < np; ++j) {
       const uint32_t sq = seq + j;
-      const int s = sq % CF::kNS;
-      const bool w = mbar_wait(&wbars[s], (sq / CF::kNS) & 1u, kWaitLimitNs);
+      const int s = sq % NS;
+      const bool w = mbar_wait(&wbars[s], (sq / NS) & 1u, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         jfail = j;
@@ -706,14 +715,18 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         __syncwarp();
       }
       const uint32_t kb_u = smem_u32(kbuf), vb_u = smem_u32(vbuf);
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      // S^T = K Q^T over d in two independent accumulator chains (even and odd
+      // 16-wide d slices), so the page's score latency is half a dependent chain
+      float c[4] = {0.f, 0.f, 0.f, 0.f}, c2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const int col = ks * 16 + a_colh;
         uint32_t a0, a1, a2, a3;
         ldsm_x4(kb_u + (col >> 6) * (kPage * 128) + swz(a_row, col & 63), a0, a1, a2, a3);
-        mma_16816(c, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+        mma_16816((ks & 1) ? c2 : c, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
       }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c[i] += c2[i];
       // mask, scale, online softmax per head (columns (lane%4)*2 and +1)
       const float s0 = key_lo < valid ? c[0] * p.scale_log2 : -INFINITY;
       const float s1 = key_lo < valid ? c[1] * p.scale_log2 : -INFINITY;
@@ -745,7 +758,7 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         acc[mt][3] *= alB;
         mma_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
       }
-      const int jn = j + CF::kNS;
+      const int jn = j + NS;
       if (jn < np) {
         if ((jn >> 5) > win) {     // next window; fetch the one after it
           ++win;
@@ -755,17 +768,17 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         }
         const int blk = __shfl_sync(0xffffffffu, bt_cur, jn & 31);
         __syncwarp();
-        if (lane == 0) decode_issue_page<D>(p, ring, wbars, sq + CF::kNS, blk, kvh);
+        if (lane == 0) decode_issue_page<D, NS>(p, ring, wbars, sq + NS, blk, kvh);
       }
     }
     if (!ok) {
       // drain copies still in flight into this warp's ring before giving up
       if (lane == 0) {
         record_error(p, POD_ERR_TIMEOUT, 3);
-        const int jend = min(np, jfail + CF::kNS);
+        const int jend = min(np, jfail + NS);
         for (int j = jfail + 1; j < jend; ++j) {
           const uint32_t sq = seq + (uint32_t)j;
-          mbar_wait(&wbars[sq % CF::kNS], (sq / CF::kNS) & 1u, kWaitLimitNs / 4);
+          mbar_wait(&wbars[sq % NS], (sq / NS) & 1u, kWaitLimitNs / 4);
         }
       }
       *abort_flag = 1;
@@ -887,8 +900,12 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
   }
 
   uint32_t tiles_done = 0, items_done = 0, seq = 0;
-  uint8_t* ring = smem + (warp < kWarpsPerCta ? warp : 0) * CF::kNS * CF::kDecStage;
-  uint64_t* wbars = &bars[kBarDecode + (warp < kWarpsPerCta ? warp : 0) * CF::kNS];
+  // decode page rings: warp w < decode_warps owns ring w (ns stages) and its ns barriers
+  const bool all_decode = p.decode_warps == kAllWarps;
+  const int dwarps = all_decode ? kAllWarps : kWarpsPerCta;
+  const int ns = all_decode ? CF::kNSAll : CF::kNS;
+  uint8_t* ring = smem + (warp < dwarps ? warp : 0) * ns * CF::kDecStage;
+  uint64_t* wbars = &bars[kBarDecode + (warp < dwarps ? warp : 0) * ns];
 
   for (int phase = 0; phase < 2; ++phase) {
     const int role = phase == 0 ? home : 1 - home;
@@ -927,7 +944,8 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
         items_done += 1;
       }
     } else {
-      if (warp < kWarpsPerCta) decode_warp<D>(p, ring, wbars, seq, sh_abort, home);
+      if (all_decode) decode_warp<D, CF::kNSAll>(p, ring, wbars, seq, sh_abort, home);
+      else if (warp < kWarpsPerCta) decode_warp<D, CF::kNS>(p, ring, wbars, seq, sh_abort, home);
       __syncthreads();
     }
   }
@@ -1254,6 +1272,7 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   prm.merge_cnt = reinterpret_cast<int32_t*>(w + pl->off_merge_cnt);
   prm.merge_in_kernel = (pl->cfg.flags & POD_FLAG_MERGE_KERNEL) ? 0 : 1;
   prm.selftest_timeout = (pl->cfg.flags & POD_FLAG_SELFTEST_TIMEOUT) ? 1 : 0;
+  prm.decode_warps = (pl->cfg.flags & POD_FLAG_DECODE_FOUR_WARPS) ? kWarpsPerCta : kAllWarps;
   if ((pl->cfg.flags & POD_FLAG_SM_PARTITION) && pl->n_pre > 0 && pl->n_dec > 0) {
     // as many SMs as the prefill items fill with every CTA of the SM, at least one, at most all
     const int64_t want = ((int64_t)pl->n_pre + pl->ctas - 1) / pl->ctas;

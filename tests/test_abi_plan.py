@@ -54,8 +54,9 @@ def _lens(w):
 def _compare(pod, Hq, Hkv, d, sms, P, KV, lens, **kw):
     ref = plan_ref(Hq, Hkv, d, sms, P, KV, lens, **kw)
     ratio = (kw.get("ratio_p", 0), kw.get("ratio_d", 0))
+    flags = pod.POD_FLAG_DECODE_FOUR_WARPS if kw.get("decode_warps", 6) == 4 else 0
     pl = pod.Plan(Hq, Hkv, d, P, KV, lens, num_sms=sms, ctas_per_sm=kw.get("ctas_per_sm", 0), ratio=ratio,
-                  max_waves=kw.get("max_waves", 0), min_chunk_pages=kw.get("min_chunk_pages", 0))
+                  max_waves=kw.get("max_waves", 0), min_chunk_pages=kw.get("min_chunk_pages", 0), flags=flags)
     pre, dec, mer = pl.tables()
     np.testing.assert_array_equal(pre, ref.prefill_items)
     np.testing.assert_array_equal(dec, ref.decode_items)
@@ -89,7 +90,8 @@ def test_c_plan_matches_plan_ref_random(pod):
         lens = [int(x) for x in rng.integers(1, 9000, size=B)]
         kw = dict(ctas_per_sm=int(rng.choice([0, 1, 2])), max_waves=int(rng.choice([0, 1, 3])),
                   min_chunk_pages=int(rng.choice([0, 1, 4, 16])),
-                  ratio_p=int(rng.choice([0, 0, 1, 2])), ratio_d=int(rng.choice([0, 0, 1, 3])))
+                  ratio_p=int(rng.choice([0, 0, 1, 2])), ratio_d=int(rng.choice([0, 0, 1, 3])),
+                  decode_warps=int(rng.choice([4, 6])))
         _compare(pod, Hkv * g, Hkv, int(rng.choice([64, 128])), int(rng.integers(1, 200)), P, C + P, lens, **kw)
 
 
@@ -113,8 +115,9 @@ def test_c_plan_rejects(pod, bad, code):
 def _compare_batched(pod, Hq, Hkv, d, sms, qo, kv, lens, **kw):
     ref = plan_ref_batched(Hq, Hkv, d, sms, qo, kv, lens, **kw)
     ratio = (kw.get("ratio_p", 0), kw.get("ratio_d", 0))
+    flags = pod.POD_FLAG_DECODE_FOUR_WARPS if kw.get("decode_warps", 6) == 4 else 0
     pl = pod.Plan(Hq, Hkv, d, qo, kv, lens, num_sms=sms, ctas_per_sm=kw.get("ctas_per_sm", 0), ratio=ratio,
-                  max_waves=kw.get("max_waves", 0), min_chunk_pages=kw.get("min_chunk_pages", 0))
+                  max_waves=kw.get("max_waves", 0), min_chunk_pages=kw.get("min_chunk_pages", 0), flags=flags)
     pre, dec, mer = pl.tables()
     np.testing.assert_array_equal(pre, ref.prefill_items)
     np.testing.assert_array_equal(dec, ref.decode_items)
@@ -141,7 +144,7 @@ def test_c_batched_plan_matches_plan_ref_random(pod):
         kv = [P + (int(rng.integers(0, 3000)) if P else int(rng.integers(0, 5))) for P in qo]
         lens = [int(x) for x in rng.integers(1, 6000, size=int(rng.integers(0, 30)))]
         kw = dict(ctas_per_sm=int(rng.choice([0, 1, 2])), max_waves=int(rng.choice([0, 1, 3])),
-                  min_chunk_pages=int(rng.choice([0, 1, 16])))
+                  min_chunk_pages=int(rng.choice([0, 1, 16])), decode_warps=int(rng.choice([4, 6])))
         _compare_batched(pod, Hkv * g, Hkv, int(rng.choice([64, 128])), int(rng.integers(1, 200)), qo, kv, lens, **kw)
 
 

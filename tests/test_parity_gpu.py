@@ -76,7 +76,7 @@ SMALL = [
 
 
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
-@pytest.mark.parametrize("flags", [0, 1], ids=["fused", "sequential"])
+@pytest.mark.parametrize("flags", [0, 1, 64, 65], ids=["fused", "sequential", "four_warps", "four_warps_sequential"])
 def test_small_batches_full_parity(env, w, flags):
     b = synth.make_batch(w)
     db, pl, ws = _run(env, b, flags=flags)
@@ -91,10 +91,12 @@ def test_small_batches_full_parity(env, w, flags):
 @pytest.mark.parametrize("kw", [dict(ctas_per_sm=1), dict(ratio=(0, 1)), dict(ratio=(1, 0)), dict(max_waves=8),
                                 dict(min_chunk_pages=1), dict(num_sms=7), dict(flags=4, max_waves=8),
                                 dict(flags=5, max_waves=8), dict(flags=16), dict(flags=16 | 4, max_waves=8),
-                                dict(flags=32)],
+                                dict(flags=32), dict(flags=64, ratio=(0, 1)), dict(flags=64 | 16),
+                                dict(flags=64 | 4, max_waves=8), dict(flags=64 | 32)],
                          ids=["one_cta", "decode_first", "prefill_first", "many_splits", "tiny_splits", "few_sms",
                               "merge_kernel", "merge_kernel_sequential", "two_streams", "two_streams_merge_kernel",
-                              "sm_partition"])
+                              "sm_partition", "four_warps_decode_first", "four_warps_two_streams",
+                              "four_warps_merge_kernel", "four_warps_sm_partition"])
 def test_knobs_keep_results(env, kw):
     w = synth.custom("knobs", 8, 2, 128, 300, 700, [16, 33, 1000, 2500, 4096], 12)
     b = synth.make_batch(w)
@@ -118,7 +120,7 @@ BATCHED = [
 
 
 @pytest.mark.parametrize("w", BATCHED, ids=lambda w: w.name)
-@pytest.mark.parametrize("flags", [0, 1, 16], ids=["fused", "sequential", "two_streams"])
+@pytest.mark.parametrize("flags", [0, 1, 16, 64], ids=["fused", "sequential", "two_streams", "four_warps"])
 def test_batched_full_parity(env, w, flags):
     b = synth.make_batch(w)
     db, pl, ws = _run(env, b, flags=flags)
@@ -160,6 +162,12 @@ def test_llama3_8b_mix_sampled(env):
     reqs = [0, 1, 7, 31, 32, 62, 63]
     db, pl, ws, b = _sampled(env, w, rows, reqs)
     assert pl.info.num_partials > 0       # the workload exercises split-KV + merge
+
+
+def test_llama3_8b_mix_sampled_four_warps(env):
+    """The same full-size batch with only warps 0-3 decoding (3-page rings)."""
+    w = synth.llama3_8b_mix()
+    _sampled(env, w, [0, 127, 128, 383, 511], [0, 1, 31, 63], flags=64)
 
 
 @pytest.mark.slow

@@ -26,7 +26,7 @@ def _plan(w, **kw):
     return plan_ref(w.num_q_heads, w.num_kv_heads, w.head_dim, SMS, P, C + P, _lens(w), **kw)
 
 
-def check_plan(pl, Hq, Hkv, P, C, lens, sms=SMS, waves=2, minc=16):
+def check_plan(pl, Hq, Hkv, P, C, lens, sms=SMS, waves=2, minc=16, dwarps=6):
     # prefill coverage: each (tile, head) once, kv_end = C + tile end
     T = -(-P // 128)
     seen = set()
@@ -67,7 +67,7 @@ def check_plan(pl, Hq, Hkv, P, C, lens, sms=SMS, waves=2, minc=16):
     pages = [-(-(k1 - k0) // PAGE) for _, _, k0, k1, *_ in pl.decode_items.tolist()]
     assert pages == sorted(pages, reverse=True)
     # cap: at most max_waves * decode warps items unless nothing splits
-    cap = waves * sms * pl.ctas_per_sm * 4
+    cap = waves * sms * pl.ctas_per_sm * dwarps
     if pl.num_partials > 0:
         assert len(pl.decode_items) <= cap
     # merge items: contiguous partial ranges covering all partials once
@@ -99,8 +99,21 @@ def test_plan_invariants_random():
         sms = int(rng.integers(1, 149))
         k = int(rng.choice([0, 1, 2]))
         waves = int(rng.choice([0, 1, 2, 3]))
-        pl = plan_ref(Hkv * g, Hkv, 128, sms, P, C + P, lens, ctas_per_sm=k, max_waves=waves)
-        check_plan(pl, Hkv * g, Hkv, P, C, lens, sms, waves or 2)
+        dw = int(rng.choice([4, 6]))
+        pl = plan_ref(Hkv * g, Hkv, 128, sms, P, C + P, lens, ctas_per_sm=k, max_waves=waves, decode_warps=dw)
+        check_plan(pl, Hkv * g, Hkv, P, C, lens, sms, waves or 2, dwarps=dw)
+
+
+def test_split_cap_counts_decode_warps():
+    """Six decode warps per CTA allow 1.5x the items of four: the cap of four warps at 3 waves."""
+    w = synth.decode_heavy_mix()
+    six = _plan(w)
+    four = _plan(w, decode_warps=4)
+    four_w3 = _plan(w, decode_warps=4, max_waves=3)
+    assert len(six.decode_items) > len(four.decode_items)
+    np.testing.assert_array_equal(six.decode_items, four_w3.decode_items)
+    with pytest.raises(PlanError):
+        _plan(w, decode_warps=5)
 
 
 def test_ratio_rules():

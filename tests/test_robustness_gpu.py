@@ -58,15 +58,16 @@ def test_expired_wait_is_reported_and_attention_still_runs(env):
     assert db.error_word(pl2, ws2) == 0
 
 
+@pytest.mark.parametrize("flags", [0, 64], ids=["six_decode_warps", "four_decode_warps"])
 @pytest.mark.parametrize("bad", [10 ** 6, -7])
-def test_out_of_range_block_id_is_reported_not_faulted(env, bad):
+def test_out_of_range_block_id_is_reported_not_faulted(env, bad, flags):
     torch, pod = env
     b = synth.make_batch(W)
     db = DeviceBatch(torch, b)
     bt = b.block_table.copy()
     bt[3, 5] = bad                     # decode request 2 (1500 tokens), page 5
     db.bt = torch.from_numpy(bt).cuda()
-    pl = db.plan(pod)
+    pl = db.plan(pod, flags=flags)
     ws = db.workspace(pl)
     pl.upload(ws)
     db.run(pod, pl, ws)
@@ -97,8 +98,9 @@ def test_lengths_that_disagree_with_the_plan_are_reported(env):
     assert db.error_word(pl, ws) == pod.POD_ERR_PLAN_MISMATCH
 
 
-@pytest.mark.parametrize("ratio", [(0, 0), (1, 0), (0, 1)], ids=["proportional", "prefill_first", "decode_first"])
-def test_schedule_trace(env, ratio):
+@pytest.mark.parametrize("ratio,extra", [((0, 0), 0), ((1, 0), 0), ((0, 1), 0), ((0, 0), 64)],
+                         ids=["proportional", "prefill_first", "decode_first", "proportional_four_warps"])
+def test_schedule_trace(env, ratio, extra):
     """Every item runs exactly once; with two CTAs per SM and a 1:1 ratio each SM
     has one prefill-home and one decode-home CTA; 1:0 and 0:1 make every CTA
     prefill-home or decode-home."""
@@ -106,7 +108,7 @@ def test_schedule_trace(env, ratio):
     w = synth.custom("trace", 32, 8, 128, 512, 2048, list(range(300, 6000, 97)), 32)
     b = synth.make_batch(w)
     db = DeviceBatch(torch, b)
-    pl = db.plan(pod, flags=pod.POD_FLAG_TRACE, ratio=ratio)
+    pl = db.plan(pod, flags=pod.POD_FLAG_TRACE | extra, ratio=ratio)
     ws = db.workspace(pl)
     pl.upload(ws)
     n = pl.info.num_prefill_items + pl.info.num_decode_items
