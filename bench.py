@@ -186,6 +186,14 @@ def cpu_oracle_time(b, decode_reqs, prefill_rows):
     return t1 - t0, t2 - t1, od, op
 
 
+def cpu_oracle_single_thread_us(b, decode_reqs, prefill_rows):
+    """The same sampled oracle run with BLAS held to one thread, scaled to the whole batch (µs)."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1, user_api="blas"):
+        td, tp, _, _ = cpu_oracle_time(b, decode_reqs, prefill_rows)
+    return extrapolate(b, decode_reqs, prefill_rows, td, tp) * 1e6
+
+
 def extrapolate(b, decode_reqs, prefill_rows, t_dec, t_pre):
     """Scale sampled oracle time to the whole batch by keys visited."""
     L = b.decode_lens.astype(np.int64)
@@ -499,7 +507,8 @@ def main():
         cpu = {"value": v, "unit": "us", "cores": blas_threads(), "kind": "oracle",
                "sample": f"every 8th decode request ({len(reqs)}) and every 8th prefill row ({len(rows)}), all "
                          f"heads; measured {td + tp:.2f} s, scaled to the whole batch by keys visited",
-               "host_cpus": os.cpu_count()}
+               "host_cpus": os.cpu_count(),
+               "single_thread_value": cpu_oracle_single_thread_us(b, reqs, rows)}
         # the oracle outputs of that sample double as a parity spot check of the timed path
         gp, gd = db.outputs()
         e_dec = np.abs(gd[reqs] - od) if od is not None else np.zeros(1)

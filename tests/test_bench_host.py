@@ -60,3 +60,11 @@ def test_plan_digest_tracks_the_tables():
     b = pod.Plan(8, 2, 128, 300, 900, [100, 2000], num_sms=148)
     c = pod.Plan(8, 2, 128, 300, 900, [100, 2001], num_sms=148)
     assert bench.plan_digest(a) == bench.plan_digest(b) != bench.plan_digest(c)
+
+
+def test_single_thread_oracle_figure_is_positive_and_scaled():
+    b = synth.make_batch(synth.tiny())
+    reqs, rows = bench.sample_sets(b, 2)
+    v = bench.cpu_oracle_single_thread_us(b, reqs, rows)
+    assert v > 0
+    assert bench.blas_threads() >= 1
