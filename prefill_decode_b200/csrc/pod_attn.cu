@@ -989,6 +989,8 @@ __global__ void __launch_bounds__(128) pod_merge_kernel(const MergeParams mp) {
 }  // namespace pod
 
 // =========================================================== host side (ABI)
+#include <atomic>
+
 using namespace pod;
 
 namespace {
@@ -1017,18 +1019,18 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 template <int D>
 int configure_kernels() {
-  static bool done[64] = {false};
+  static std::atomic<bool> done[64];   // per device; setting the attributes twice is harmless
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 64 && done[dev]) return POD_OK;
+  if (dev < 64 && done[dev].load(std::memory_order_acquire)) return POD_OK;
   e = cudaFuncSetAttribute(pod_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemAlloc);
   if (e != cudaSuccess) return cuda_fail(e);
   // two CTAs of ~113 KB need the whole 228 KB shared-memory carveout on every launch
   e = cudaFuncSetAttribute(pod_attn_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
                            (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 64) done[dev] = true;
+  if (dev < 64) done[dev].store(true, std::memory_order_release);
   return POD_OK;
 }
 
@@ -1050,10 +1052,21 @@ int side_stream(SideStream** out) {
   std::lock_guard<std::mutex> g(make);
   SideStream& s = sides[dev];
   if (!s.stream) {
-    e = cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
-    if (e != cudaSuccess) return cuda_fail(e);
+    // publish the set only when all three objects exist; release what a failed attempt made
+    cudaStream_t st = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      if (join) cudaEventDestroy(join);
+      if (fork) cudaEventDestroy(fork);
+      if (st) cudaStreamDestroy(st);
+      return cuda_fail(e);
+    }
+    s.fork = fork;
+    s.join = join;
+    s.stream = st;
   }
   *out = &s;
   return POD_OK;
