@@ -218,3 +218,39 @@ def test_c_plan_rejects_too_many_heads_and_overflowing_work(pod):
     assert e.value.status == pod.POD_ERR_INVALID_ARG
     # the largest head count still plans, and agrees with the planner of record
     _compare_batched(pod, 4096, 512, 128, 148, [128], [1 << 20], [100])
+
+
+def test_c_planner_matches_plan_ref_property(pod):
+    """Property check over generated batches (hypothesis): the C planner and the
+    written rule agree on every table, or both reject the batch."""
+    from hypothesis import given, settings, HealthCheck, strategies as st
+
+    chunk = st.tuples(st.sampled_from([0, 1, 2, 63, 64, 65, 127, 128, 129, 255, 256, 257, 1000]),
+                      st.integers(0, 5000))
+    batch = st.fixed_dictionaries(dict(
+        Hkv=st.sampled_from([1, 2, 3, 8]), g=st.integers(1, 8), d=st.sampled_from([64, 128]),
+        sms=st.integers(1, 300), chunks=st.lists(chunk, max_size=5),
+        lens=st.lists(st.integers(1, 40000), max_size=40),
+        ctas=st.sampled_from([0, 1, 2]), waves=st.integers(0, 4), minc=st.integers(0, 40),
+        rp=st.integers(0, 3), rd=st.integers(0, 3), dw=st.sampled_from([4, 6])))
+
+    @settings(max_examples=150, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+    @given(batch)
+    def check(x):
+        qo = [P for P, _ in x["chunks"]]
+        kv = [P + C if P else C % 3 for P, C in x["chunks"]]
+        kw = dict(ctas_per_sm=x["ctas"], max_waves=x["waves"], min_chunk_pages=x["minc"],
+                  ratio_p=x["rp"], ratio_d=x["rd"], decode_warps=x["dw"])
+        try:
+            ref = plan_ref_batched(x["Hkv"] * x["g"], x["Hkv"], x["d"], x["sms"], qo, kv, x["lens"], **kw)
+        except PlanError:
+            ref = None
+        if ref is None:
+            with pytest.raises(pod.PodError):
+                pod.Plan(x["Hkv"] * x["g"], x["Hkv"], x["d"], qo, kv, x["lens"], num_sms=x["sms"],
+                         ctas_per_sm=x["ctas"], ratio=(x["rp"], x["rd"]), max_waves=x["waves"],
+                         min_chunk_pages=x["minc"], flags=pod.POD_FLAG_DECODE_FOUR_WARPS if x["dw"] == 4 else 0)
+            return
+        _compare_batched(pod, x["Hkv"] * x["g"], x["Hkv"], x["d"], x["sms"], qo, kv, x["lens"], **kw)
+
+    check()
