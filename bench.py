@@ -17,7 +17,7 @@ L2, so no flush is needed between steps.
 With N > 1 (torchrun, one process per GPU) every rank runs an independent
 replica of the batch (the path has no exchange step); the reported time is the
 max over ranks.  ``--impl reference`` times the CPU float64 oracle instead (on
-rank 0 only), on a bounded sample of the same batch, extrapolated per batch.
+rank 0 only): each step is one oracle pass over the whole batch.
 """
 from __future__ import annotations
 
@@ -227,26 +227,37 @@ def sample_sets(b, frac_den: int):
     return reqs, rows
 
 
+def fp8_alg_bytes(info, w) -> int:
+    """Algorithmic bytes of a run whose decodes read e4m3 K/V (1 byte per element) and whose
+    prefill requests read bf16 K/V: decode K/V + prefill K/V + Q + O."""
+    dec_tokens = info.decode_flops // (4 * w.head_dim * w.num_q_heads)
+    dec_kv16 = 4 * w.head_dim * w.num_kv_heads * dec_tokens
+    return int(info.kv_bytes - dec_kv16 // 2 + info.qo_bytes)
+
+
 # ------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
+    """The reference arm: the float64 oracle over the WHOLE batch per step (every decode
+    request and every prefill row, all heads), on the host cores, rank 0 only."""
     if rank != 0:
         return 0
     w = synth.NAMED[args.workload]()
     b = synth.make_batch(w)
-    reqs, rows = sample_sets(b, 8)
+    reqs, rows = list(range(w.num_decode)), list(range(w.prefill_rows))
     times = []
     for i in range(args.warmup + args.steps):
         td, tp, _, _ = cpu_oracle_time(b, reqs, rows)
         if i >= args.warmup:
-            times.append(extrapolate(b, reqs, rows, td, tp) * 1e6)
+            times.append((td + tp) * 1e6)
     v = float(np.mean(times))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(w, b, "oracle"),
             "cpu_baseline": {"value": v, "unit": "us", "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"every 8th decode request ({len(reqs)}) and every 8th prefill row "
-                                       f"({len(rows)}), all heads; time scaled to the whole batch by keys visited"},
+                             "host_cpus": os.cpu_count(),
+                             "sample": f"the whole batch every step: all {len(reqs)} decode requests and all "
+                                       f"{len(rows)} prefill rows, every head; no extrapolation"},
             "e2e": {"value": v, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -271,13 +282,20 @@ def run_sweep(args):
     from prefill_decode_b200 import build
     build.build()
     import prefill_decode_b200 as pod
-    from tests.podrun import DeviceBatch
+    from prefill_decode_b200.device_batch import DeviceBatch
     peaks, peak_src = load_peaks()
     names = args.sweep.split(",") if args.sweep not in ("1", "all") else None
     wls = [synth.NAMED[n]() for n in sorted(synth.NAMED)] + synth.sweep_points()
     if names:
         wls = [w for w in wls if w.name in names]
     stream = torch.cuda.current_stream()
+    gpu_id = "0"
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(0).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
     for w in wls:
         db = DeviceBatch.generated_on_device(torch, w)
         res = {"workload": w.name, "values": "torch.Generator(cuda, seed) normals; layout from synth"}
@@ -287,38 +305,66 @@ def run_sweep(args):
             arms += (("fused_1_1", dict(ratio=(1, 1))), ("fused_1_0", dict(ratio=(1, 0))),
                      ("sm_partition", dict(flags=pod.POD_FLAG_SM_PARTITION)),
                      ("four_decode_warps", dict(flags=pod.POD_FLAG_DECODE_FOUR_WARPS)))
+        if args.sweep_splits:
+            arms += (("split_unlimited", dict(flags=pod.POD_FLAG_PREFILL_SPLIT_UNLIMITED)),
+                     ("split_never", dict(max_prefill_splits=1)),
+                     ("sequential_split_unlimited",
+                      dict(flags=pod.POD_FLAG_SEQUENTIAL | pod.POD_FLAG_PREFILL_SPLIT_UNLIMITED)))
+        if args.sweep_fp8 and w.num_decode:
+            db.fp8_on_device()
+            arms += (("fused_fp8_kv", dict(_fp8=True)),)
         for mode, kw in arms:
+            kw = dict(kw)
+            use8 = kw.pop("_fp8", False)
             pl = db.plan(pod, **kw)
             ws = db.workspace(pl)
             pl.upload(ws, stream)
-            ev = [(pod.Event(), pod.Event()) for _ in range(args.steps)]
+            run = (lambda: db.run_fp8(pod, pl, ws, stream=stream)) if use8 else (lambda: db.run(pod, pl, ws, stream=stream))
             for _ in range(args.warmup):
-                db.run(pod, pl, ws, stream=stream)
+                run()
             torch.cuda.synchronize()
+            # enough steps for the timed window to span a few clock samples (>= 0.4 s), at most 4000
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for i in range(args.steps):
-                pl.set_events(ev[i][0].handle, ev[i][1].handle)
-                db.run(pod, pl, ws, stream=stream)
+            for _ in range(5):
+                run()
             e1.record(stream)
             torch.cuda.synchronize()
+            est_s = e0.elapsed_time(e1) / 5e3
+            steps = int(min(4000, max(args.steps, 0.4 / max(est_s, 1e-6))))
+            ev = [(pod.Event(), pod.Event()) for _ in range(steps)]
+            t_w0 = time.time()
+            e0.record(stream)
+            for i in range(steps):
+                pl.set_events(ev[i][0].handle, ev[i][1].handle)
+                run()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            t_w1 = time.time()
             pl.set_events(None, None)
             info = pl.info
-            step_us = e0.elapsed_time(e1) * 1e3 / args.steps
+            step_us = e0.elapsed_time(e1) * 1e3 / steps
             kern_us = float(np.mean([a.elapsed_ms(c) for a, c in ev])) * 1e3
-            t_hbm = (info.kv_bytes + info.qo_bytes) / (peaks["hbm_gbs"] * 1e9) * 1e6
+            alg_bytes = fp8_alg_bytes(info, w) if use8 else info.kv_bytes + info.qo_bytes
+            t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6
             t_tc = info.prefill_flops / (peaks["bf16_tflops"] * 1e12) * 1e6
-            res[mode] = {"step_us": step_us, "kernel_us": kern_us, "roofline_us": max(t_hbm, t_tc),
-                         "frac_step": max(t_hbm, t_tc) / step_us, "bound": "hbm" if t_hbm >= t_tc else "tensor",
-                         "hbm_GBps": (info.kv_bytes + info.qo_bytes) / (kern_us * 1e-6) / 1e9,
+            ck = sampler.summary(t_w0, t_w1)
+            res[mode] = {"steps": steps, "step_us": step_us, "kernel_us": kern_us, "roofline_us": max(t_hbm, t_tc),
+                         "frac_step": max(t_hbm, t_tc) / step_us, "frac_kernel": max(t_hbm, t_tc) / kern_us,
+                         "bound": "hbm" if t_hbm >= t_tc else "tensor", "algorithmic_bytes": int(alg_bytes),
+                         "hbm_GBps": alg_bytes / (kern_us * 1e-6) / 1e9,
                          "prefill_TFLOPs": info.prefill_flops / (kern_us * 1e-6) / 1e12,
-                         "error_word": db.error_word(pl, ws)}
+                         "prefill_items": info.num_prefill_items, "prefill_partials": info.num_prefill_partials,
+                         "error_word": db.error_word(pl, ws),
+                         "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"],
+                                    "reasons": ck["reasons"], "samples": ck["samples"]}}
         res["speedup_vs_sequential"] = res["sequential"]["step_us"] / res["fused"]["step_us"]
         res["speedup_vs_two_streams"] = res["two_streams"]["step_us"] / res["fused"]["step_us"]
         res["peaks"] = peak_src
         print(json.dumps(res), flush=True)
         del db
         torch.cuda.empty_cache()
+    sampler.stop()
     return 0
 
 
@@ -332,15 +378,20 @@ def main():
     ap.add_argument("--workload", default="llama3_8b_mix", choices=sorted(synth.NAMED))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 KV-cache arm")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--sweep-ratios", action="store_true",
                     help="sweep mode: also time the fused kernel at forced role ratios 1:1 and 1:0")
+    ap.add_argument("--sweep-splits", action="store_true",
+                    help="sweep mode: also time the prefill KV split without its co-located limit and without any split")
+    ap.add_argument("--sweep-fp8", action="store_true",
+                    help="sweep mode: also time the fused kernel with the decode requests on an e4m3 KV cache")
     ap.add_argument("--sweep", default=None,
                     help="'all' or comma-separated workload names: per-workload table lines instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.sweep:
-        args.steps = min(args.steps, 200)
+        args.steps = min(args.steps, 200)   # a floor: each arm runs for at least 0.4 s of steps
         return run_sweep(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -355,7 +406,7 @@ def main():
     from prefill_decode_b200 import build
     build.build()
     import prefill_decode_b200 as pod
-    from tests.podrun import DeviceBatch
+    from prefill_decode_b200.device_batch import DeviceBatch
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -422,7 +473,9 @@ def main():
     for name, kw in (("two_streams", dict(flags=pod.POD_FLAG_TWO_STREAMS)),
                      ("sm_partition", dict(flags=pod.POD_FLAG_SM_PARTITION)),
                      ("decode_four_warps", dict(flags=pod.POD_FLAG_DECODE_FOUR_WARPS)),
-                     ("prefill_first_1_0", dict(ratio=(1, 0))), ("decode_first_0_1", dict(ratio=(0, 1)))):
+                     ("prefill_first_1_0", dict(ratio=(1, 0))), ("decode_first_0_1", dict(ratio=(0, 1))),
+                     ("prefill_split_unlimited", dict(flags=pod.POD_FLAG_PREFILL_SPLIT_UNLIMITED)),
+                     ("prefill_split_never", dict(max_prefill_splits=1))):
         pl_a = db.plan(pod, **kw)
         ws_a = db.workspace(pl_a)
         pl_a.upload(ws_a, stream)
@@ -432,6 +485,44 @@ def main():
                            "kernels_us": max_over_ranks(float(np.mean(a_kern)) * 1e3),
                            "error_word": db.error_word(pl_a, ws_a)}
         del ws_a
+    # the decode requests on an e4m3 copy of the cache (pod_attn_run_fp8kv), same plan and timing
+    fp8_arm = None
+    if w.num_decode and not args.no_fp8:
+        db.fp8_on_device()
+        ws8 = db.workspace(fused)
+        fused.upload(ws8, stream)
+        ev8 = [(pod.Event(), pod.Event()) for _ in range(k_abl)]
+        for _ in range(args.warmup):
+            db.run_fp8(pod, fused, ws8, stream=stream)
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(k_abl):
+            fused.set_events(ev8[i][0].handle, ev8[i][1].handle)
+            db.run_fp8(pod, fused, ws8, stream=stream)
+        f1.record(stream)
+        barrier()
+        fused.set_events(None, None)
+        k8_us = max_over_ranks(float(np.mean([a.elapsed_ms(c) for a, c in ev8])) * 1e3)
+        b8 = fp8_alg_bytes(fused.info, w)
+        fp8_arm = {"step_us": max_over_ranks(f0.elapsed_time(f1) * 1e3 / k_abl), "kernel_us": k8_us,
+                   "algorithmic_bytes": b8, "hbm_GBps": b8 / (k8_us * 1e-6) / 1e9,
+                   "error_word": db.error_word(fused, ws8),
+                   "note": "decode K/V as e4m3 codes with one fp32 scale per kv head (made on the GPU from the "
+                           "bf16 pools), prefill K/V bf16; bytes = decode K/V at 1 byte + prefill K/V at 2 + Q + O"}
+        # parity spot check of the e4m3 run against the float64 oracle on the same codes
+        from oracle import attention as A8, fp8 as F8
+        reqs8 = [0, w.num_decode // 2, w.num_decode - 1]
+        K8 = F8.dequant_pool(db.k8.cpu().numpy(), db.k_scale.cpu().numpy())
+        V8 = F8.dequant_pool(db.v8.cpu().numpy(), db.v_scale.cpu().numpy())
+        ref8 = A8.attend_decode(b.q_decode, K8, V8, b.block_table, b.kv_lens, b.scale, w.num_kv_heads,
+                                requests=reqs8, first_row=b.num_prefill)
+        got8 = db.o_dec.float().cpu().numpy()[reqs8]
+        fp8_arm["parity_sample"] = {"requests": reqs8, "max_abs": float(np.abs(got8 - ref8).max()),
+                                    "mean_abs": float(np.abs(got8 - ref8).mean())}
+        del K8, V8, ws8
+        db.run(pod, fused, ws, stream=stream)   # leave the bf16 outputs for the parity sample below
+        torch.cuda.synchronize()
     sampler.stop()
     err_word = db.error_word(fused, ws)
 
@@ -501,20 +592,24 @@ def main():
     cpu = None
     parity = None
     if not args.no_cpu_baseline:
-        reqs, rows = sample_sets(b, 8)
+        # the oracle as it stands over the whole batch (all cores), and a single-thread figure from every
+        # 8th request and row scaled by keys visited; the full-batch outputs double as a parity check
+        reqs, rows = list(range(w.num_decode)), list(range(w.prefill_rows))
         td, tp, od, op = cpu_oracle_time(b, reqs, rows)
-        v = extrapolate(b, reqs, rows, td, tp) * 1e6
-        cpu = {"value": v, "unit": "us", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"every 8th decode request ({len(reqs)}) and every 8th prefill row ({len(rows)}), all "
-                         f"heads; measured {td + tp:.2f} s, scaled to the whole batch by keys visited",
+        s_reqs, s_rows = sample_sets(b, 8)
+        cpu = {"value": (td + tp) * 1e6, "unit": "us", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"the whole batch: all {len(reqs)} decode requests and all {len(rows)} prefill rows, "
+                         f"every head, one pass ({td + tp:.2f} s)",
                "host_cpus": os.cpu_count(),
-               "single_thread_value": cpu_oracle_single_thread_us(b, reqs, rows)}
-        # the oracle outputs of that sample double as a parity spot check of the timed path
+               "single_thread_value": cpu_oracle_single_thread_us(b, s_reqs, s_rows),
+               "single_thread_sample": f"every 8th decode request ({len(s_reqs)}) and prefill row "
+                                       f"({len(s_rows)}) with BLAS on one thread, scaled by keys visited"}
         gp, gd = db.outputs()
-        e_dec = np.abs(gd[reqs] - od) if od is not None else np.zeros(1)
-        e_pre = np.abs(gp[rows] - op) if op is not None else np.zeros(1)
+        e_dec = np.abs(gd - od) if od is not None else np.zeros(1)
+        e_pre = np.abs(gp - op) if op is not None else np.zeros(1)
         parity = {"max_abs": float(max(e_dec.max(), e_pre.max())),
                   "mean_abs": float(np.concatenate([e_dec.ravel(), e_pre.ravel()]).mean()),
+                  "elements": int(e_dec.size + e_pre.size),
                   "tolerance": {"max_abs": 2e-2, "mean_abs": 2e-3}}
 
     line = {
@@ -525,7 +620,8 @@ def main():
         "fused_roofline": {"t_tensor_us": t_tc_us, "t_hbm_us": t_hbm_us, "t_roofline_us": max(t_tc_us, t_hbm_us),
                            "frac_step": max(t_tc_us, t_hbm_us) / us, "frac_kernel": max(t_tc_us, t_hbm_us) / kern_us,
                            "peaks": f"{peak_src}: HBM {peaks['hbm_gbs']} GB/s, bf16 {peaks['bf16_tflops']} TFLOP/s"},
-        "roofline": {"kernel": "pod_attn_kernel<128> (fused persistent)", "bound": bound, "achieved": achieved,
+        "roofline": {"kernel": f"pod::pod_attn_kernel<{w.head_dim}> (fused persistent)", "bound": bound,
+                     "achieved": achieved,
                      "peak": peak, "unit": unit, "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": traffic, "algorithmic_bytes": int(alg_bytes),
                      "algorithmic_flops_prefill": int(info.prefill_flops), "kernel_us": kern_us},
@@ -534,13 +630,21 @@ def main():
                           note="two_streams = prefill-only and decode-only kernels on concurrent streams; "
                                "sm_partition = roles by SM id instead of per-SM tickets; "
                                "decode_four_warps = only 4 of a decoding CTA's 6 warps run decode items (deeper page rings); "
-                               "x_first = ratio p:d forced so every CTA starts on that role"),
+                               "x_first = ratio p:d forced so every CTA starts on that role; "
+                               "prefill_split_unlimited = the prefill KV split fills every CTA slot (the "
+                               "co-located-decode limit for <= 1536 prefill tokens off); prefill_split_never = "
+                               "no prefill KV split"),
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
+        "launches_note": "per step: one pod_attn_kernel launch (split-KV rows merged inside it) after one "
+                         "cudaMemsetAsync of the workspace counters",
         "plan": {"prefill_items": info.num_prefill_items, "decode_items": info.num_decode_items,
                  "merge_items": info.num_merge_items, "chunk_pages": info.chunk_pages,
                  "ctas_per_sm": info.ctas_per_sm, "ratio": [info.ratio_prefill, info.ratio_decode],
-                 "grid": info.grid},
+                 "grid": info.grid, "prefill_partials": info.num_prefill_partials},
         "device_error_word": err_word, "parity_sample": parity,
+        "fp8_kv": dict(fp8_arm, frac_of_hbm_peak=fp8_arm["hbm_GBps"] / peaks["hbm_gbs"],
+                       t_roofline_us=max(fp8_arm["algorithmic_bytes"] / (peaks["hbm_gbs"] * 1e3), t_tc_us))
+        if fp8_arm else None,
     }
     if world > 1:
         dist.barrier()

@@ -86,6 +86,9 @@ enum {
                                           (page rings 3 deep for d = 128, 4 for d = 64) and the plan's
                                           split cap counts 4 decode warps per CTA; by default all 6 warps
                                           decode (the MMA and TMA warps too; rings 2 / 3 deep) */
+#define POD_FLAG_PREFILL_SPLIT_UNLIMITED 128u /* ablation: the prefill KV split fills every CTA slot even
+                                                 when a short prefill (<= 1536 tokens) shares the batch
+                                                 with decode work (the plan rule's co-located limit off) */
 
 typedef struct pod_attn_config {
   int32_t num_q_heads;      /* Hq, 1..4096 */
@@ -98,13 +101,15 @@ typedef struct pod_attn_config {
   int32_t ratio_decode;
   int32_t max_waves;        /* split-KV cap in waves of decode warps; 0 = 2 */
   int32_t min_chunk_pages;  /* smallest split, in pages; 0 = 16 */
+  int32_t max_prefill_splits; /* KV pieces per prefill item: 0 = the plan rule (at most 16), 1 = never
+                                 split the prefill, 2..16 = the rule capped at this many */
   uint32_t flags;           /* POD_FLAG_* */
 } pod_attn_config;
 
 typedef struct pod_attn_plan pod_attn_plan_t;
 
 typedef struct pod_attn_plan_info {
-  int32_t num_prefill_items;  /* (128-row query tile, query head) units */
+  int32_t num_prefill_items;  /* (128-row query tile, query head, key range) units */
   int32_t num_decode_items;   /* (request, kv head, key range) units */
   int32_t num_merge_items;    /* (request, kv head) rows with more than one split */
   int32_t num_partials;       /* split partial results held in the workspace */
@@ -123,15 +128,57 @@ typedef struct pod_attn_plan_info {
   int64_t table_bytes;        /* bytes pod_attn_upload copies host -> device */
   int32_t num_prefill_requests; /* NP: block-table / kv_lens rows 0..NP-1; decodes follow */
   int32_t num_prefill_rows;     /* sum_i P_i: rows of q_prefill / o_prefill */
+  int32_t num_prefill_partials; /* KV pieces of split prefill items (partials in the workspace) */
+  int32_t num_prefill_merge_items; /* prefill items cut into more than one KV piece */
+  int64_t rescale_count_offset; /* byte offset of an int32 in the workspace that counts, with
+                                   POD_FLAG_TRACE, the prefill softmax warps that rescaled O because
+                                   a row max grew by more than 2^8 (diagnostic; 0 without the flag) */
 } pod_attn_plan_info;
 
-/* Build the schedule for one hybrid batch on the host (no device work).
+/* The plan rule.  The sources describe the knobs (explainer "How
+ * POD-Attention overlaps prefill and decode": 2 threadblocks per SM, KV splits
+ * capped at two full waves, CTAs in proportion to the prefill:decode mix;
+ * FlashInfer PR "Limit kv split when prefill tokens <= 1536": the prefill's
+ * split count leaves room for co-located decode CTAs) but give no formula;
+ * this is the library's own rule, in integers throughout:
+ *  - k = ctas_per_sm (0 -> 2); grid = num_sms * k.
+ *  - Base prefill items: for request i (P_i rows over C_i earlier tokens), for
+ *    query tile t = ceil(P_i/128)-1 .. 0, for head h: (q0 = 128 t, h,
+ *    kv_end = C_i + min(128 (t+1), P_i), i) with n = ceil(kv_end/64) key tiles.
+ *  - Decode split: cap = max_waves (0 -> 2) * num_sms * k * decode warps per
+ *    CTA (6; 4 with POD_FLAG_DECODE_FOUR_WARPS); pages_r = ceil(L_r/16);
+ *    c = max(min_chunk_pages (0 -> 16), ceil(Hkv sum pages_r / cap)), then
+ *    c += 1 while c < max pages_r and Hkv sum ceil(pages_r / c) > cap.
+ *    Request r is cut into S_r = ceil(pages_r / c) splits; split s covers
+ *    pages [floor(s pages_r / S_r), floor((s+1) pages_r / S_r)).  Decode items
+ *    are ordered by (pages descending, r, kv head, s); merge items follow
+ *    (r, kv head) order; partial indices run over the split rows' items in
+ *    (r, kv head, s) order.
+ *  - Ticket ratio p:d: explicit ratios reduced by their gcd (a zero side gives
+ *    1:0 or 0:1).  Otherwise 0:1 without prefill, 1:0 without decode, else
+ *    cost_pre = prefill_flops, cost_dec = 248 * kv bytes of the decodes (248 =
+ *    B200 tensor FLOP/s per HBM byte/s), tot = cost_pre + cost_dec,
+ *    n_p = floor((2 k cost_pre + tot) / (2 tot)) clamped to [1, k-1] (k = 1:
+ *    n_p = 1), and n_p = k when 2 cost_pre >= tot; p:d = n_p : k - n_p reduced.
+ *  - Prefill KV split: h_p = #{t in [0,k): t mod (p+d) < p}; limited = there
+ *    are decodes and sum_i P_i <= 1536 and POD_FLAG_PREFILL_SPLIT_UNLIMITED is
+ *    off; slots = num_sms * (limited ? max(h_p, 1) : k).  With n0 base items:
+ *    if max_prefill_splits == 1 or n0 == 0 or n0 >= slots, nothing is split;
+ *    else tau = max(8, ceil(sum n / slots)) and an item of n tiles gets
+ *    S = min(smax, max(1, floor(n / tau))) pieces (smax = max_prefill_splits
+ *    if >= 2, else 16), piece s covering key tiles [floor(s n/S),
+ *    floor((s+1) n/S)).  Every piece spans at least 8 tiles.  Partial indices
+ *    run over the pieces of split items in base-item order; prefill merge
+ *    items (first partial, S) follow base-item order; all pieces are then
+ *    stably ordered by key count, longest first.
+ * The test oracle restates the same rule and the tests compare the two plans
+ * bit for bit.
+ *
+ * Build the schedule for one hybrid batch on the host (no device work).
  * One prefill request: prefill_qo_len = P (0 = no prefill); prefill_kv_len = C + P
  * (ignored if P == 0); it owns block-table / kv_lens row 0 even when P == 0,
  * and decode request r owns row 1 + r.  decode_kv_lens = host array of B
- * lengths, each >= 1.  The work items, the split-KV partition and the ticket
- * ratio follow the rule documented in oracle/plan_ref.py (the sources fix no
- * formula).  On success *plan_out owns a new plan and *workspace_bytes_out
+ * lengths, each >= 1.  On success *plan_out owns a new plan and *workspace_bytes_out
  * (nullable) receives the device workspace size that pod_attn_upload /
  * pod_attn_run need.  Same as pod_attn_plan_batched with one prefill request.
  * Errors: POD_ERR_INVALID_ARG (also when a work count of pod_attn_plan_info
@@ -158,13 +205,20 @@ int pod_attn_plan_batched(const pod_attn_config* cfg, int32_t num_prefill, const
 int pod_attn_plan_get_info(const pod_attn_plan_t* plan, pod_attn_plan_info* info);
 
 /* Host copies of the work tables, for bit-exact checks; any pointer may be null.
- *   prefill_items int32 [num_prefill_items, 4]: q0 (row within its request), q_head,
- *                                               kv_end, prefill request
+ *   prefill_items int32 [num_prefill_items, 8]: q0 (row within its request), q_head,
+ *                                               kv_end, prefill request, first and end key
+ *                                               tile of the piece (64 keys per tile),
+ *                                               partial (-1 = unsplit), prefill merge item
  *   decode_items  int32 [num_decode_items, 8]:  r, kv_head, k0, k1, partial (-1 = unsplit),
  *                                               merge item (-1 = unsplit), splits of the row, 0
  *   merge_items   int32 [num_merge_items, 4]:   r, kv_head, first_partial, num_splits */
 int pod_attn_plan_tables(const pod_attn_plan_t* plan, int32_t* prefill_items,
                          int32_t* decode_items, int32_t* merge_items);
+
+/* Copy the prefill merge table (host int32 [num_prefill_merge_items, 4]: first
+ * partial, pieces, 0, 0) into `out` (nullable = skip).  Errors:
+ * POD_ERR_INVALID_ARG (null plan). */
+int pod_attn_plan_prefill_merges(const pod_attn_plan_t* plan, int32_t* out);
 
 /* Copy the prefill request table (host int32 [num_prefill_requests, 4]: first
  * row of the request in q_prefill, P_i, C_i, 0) into `out` (nullable = skip).
@@ -182,9 +236,10 @@ int pod_attn_upload(const pod_attn_plan_t* plan, void* workspace, size_t workspa
  * merge counters in the workspace, launch the persistent fused kernel (or, with
  * POD_FLAG_SEQUENTIAL in the plan's config, the prefill-only then decode-only
  * kernels; with POD_FLAG_TWO_STREAMS, the two on concurrent streams, the call
- * still completing in `stream` order).  Split-KV partials are merged by the warp that finishes a row's
- * last split (a completion counter, no waiting), or, with POD_FLAG_MERGE_KERNEL,
- * by the LSE merge kernel launched afterwards.  Asynchronous.
+ * still completing in `stream` order).  Decode split-KV partials are merged by the warp that finishes a
+ * row's last split (a completion counter, no waiting), or, with POD_FLAG_MERGE_KERNEL,
+ * by the LSE merge kernel launched afterwards; the KV pieces of a split prefill item
+ * are always merged by the CTA that finishes the item's last piece.  Asynchronous.
  * q/k/v/o pointers: device, 16-byte aligned; q_prefill / o_prefill hold the
  * prefill requests' rows one after another ([sum_i P_i, Hq, d]); unused sides
  * (no prefill rows, or B == 0) may be null.  block_table (device int32, row
@@ -202,6 +257,35 @@ int pod_attn_run(const pod_attn_plan_t* plan,
                  void* o_prefill, void* o_decode,
                  void* workspace, size_t workspace_bytes,
                  int32_t* trace, void* stream);
+
+/* pod_attn_run with the decode requests reading an FP8 (e4m3) copy of the
+ * paged cache: the KV bytes a decode streams are halved, which is the lever
+ * the blog post "Prefill vs. Decode GPU Utilization Imbalance" names for the
+ * bandwidth-bound decode ("Quantization and compression as a lever on both the
+ * bandwidth and capacity problem").  The prefill requests keep reading the
+ * bf16 pools (k_cache / v_cache, as in pod_attn_run; unused and nullable when
+ * the plan has no prefill rows).
+ *   k_cache_fp8 / v_cache_fp8  device uint8 [num_blocks_fp8, Hkv, 16, d], 16-byte
+ *               aligned, e4m3 codes (1 sign, 4 exponent bits with bias 7, 3
+ *               mantissa bits; no infinity, S.1111.111 is NaN); decode request r
+ *               reads page block_table[NP + r][j / 16] of these pools.
+ *   k_scale / v_scale  device float32 [Hkv]: the value of a stored code c of kv
+ *               head h is k_scale[h] * e4m3(c) (v_scale for V).
+ * Scores and P.V run on f16 tensor-core operands: e4m3 codes convert exactly,
+ * and q_decode (bf16) is converted to f16, so its entries must lie within the
+ * f16 range (|q| < 65504).  Slots past a request's length may hold any code,
+ * NaN included (masked keys get no weight, masked V rows are zeroed).
+ * Everything else (plan, workspace, flags, trace, errors) is as pod_attn_run. */
+int pod_attn_run_fp8kv(const pod_attn_plan_t* plan,
+                       const void* q_prefill, const void* q_decode,
+                       const void* k_cache, const void* v_cache, int64_t num_blocks,
+                       const void* k_cache_fp8, const void* v_cache_fp8, int64_t num_blocks_fp8,
+                       const float* k_scale, const float* v_scale,
+                       const int32_t* block_table, int32_t block_table_stride,
+                       const int32_t* kv_lens, float scale,
+                       void* o_prefill, void* o_decode,
+                       void* workspace, size_t workspace_bytes,
+                       int32_t* trace, void* stream);
 
 /* Record `ev_start` / `ev_stop` (cudaEvent_t, nullable) on the stream around the
  * main attention kernel(s) of every later pod_attn_run with this plan (the
@@ -226,11 +310,15 @@ int pod_attn_event_elapsed_ms(void* ev_start, void* ev_stop, float* ms_out);
  * POD_STATIC_SCRATCH_BYTES that every GPU which loads the library holds until
  * the process exits; it allocates nothing.  Arguments, layouts and the async
  * behaviour are those of pod_attn_run (no trace).
- *  - The first call on a device looks up the array's device address for that
- *    device (cudaGetSymbolAddress); make that first call before any stream
+ *  - Every call looks up the array's device address in the current context
+ *    (cudaGetSymbolAddress), so the address stays right after cudaDeviceReset
+ *    or in another context.  The first call in a context also loads the
+ *    library's device code there; make that first call before any stream
  *    capture.
- *  - Every call re-copies the plan's tables into the array and zeroes its
- *    counters; the array keeps the last call's contents otherwise.
+ *  - Every call re-copies the plan's tables (pod_attn_plan_info.table_bytes)
+ *    into the array from the plan's pageable host copy, which can hold the
+ *    host thread for the length of that copy, and zeroes the counters; the
+ *    array keeps the last call's contents otherwise.
  *  - All calls on a device share the one array: calls that overlap on the GPU
  *    (other streams, other host threads) race and corrupt each other.
  *    Serialise them, e.g. on one stream.

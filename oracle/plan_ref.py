@@ -11,18 +11,38 @@ plan is therefore unpinned by the sources; tests pin it by invariants.
 Rule
   Validation: Hq % Hkv == 0, Hq <= 4096; g = Hq/Hkv in 1..8; d in {64, 128}; page == 16;
     1 <= num_sms <= 512; ctas_per_sm in {0 (auto = 2), 1, 2}; ratios >= 0;
-    max_waves >= 0 (0 = 2); min_chunk_pages >= 0 (0 = 16); P >= 0;
+    max_waves >= 0 (0 = 2); min_chunk_pages >= 0 (0 = 16); 0 <= prefill_splits <= 16
+    (0 = the rule below, 1 = never split the prefill); P >= 0;
     if P > 0: P <= prefill_kv_len <= 2^24; 0 <= B <= 65536; 1 <= L_r <= 2^24;
     sum_r L_r <= 2^31 - 1; every work count reported (4 d Hq sum of keys seen
     over prefill rows, 4 d Hq sum L_r, 4 d Hkv K/V tokens, 4 d Hq Q/O rows)
     fits int64.
   Prefill requests i = 0 .. NP-1 (chunk P_i over C_i = kv_i - P_i earlier
-    tokens; the one-prefill form is NP = 1, P_0 = P).  Prefill items (one
+    tokens; the one-prefill form is NP = 1, P_0 = P).  Base prefill items (one
     128-row query tile of one query head each): for i, for t = T_i-1 .. 0
     (T_i = ceil(P_i/128)), for h = 0 .. Hq-1: (q0 = 128 t, h,
-    kv_end = C_i + min(128 (t+1), P_i), request i); then stably sorted by
-    kv_end, longest first.  Prefill request table (q_start_i = P_0 + .. +
-    P_{i-1}, P_i, C_i, 0).
+    kv_end = C_i + min(128 (t+1), P_i), request i), n = ceil(kv_end / 64)
+    key tiles.  Prefill request table (q_start_i = P_0 + .. + P_{i-1}, P_i,
+    C_i, 0).
+  Prefill KV split (after the ratio below; FlashInfer PR "Limit kv split when
+    prefill tokens <= 1536": the prefill's split count leaves room for the
+    decode CTAs co-located on the same SMs while the prefill is short):
+    h_p = number of t in 0 .. k-1 with t mod (p+d) < p (prefill-home CTAs
+    per SM); limited = (B > 0 and sum_i P_i <= 1536 and the unlimited
+    ablation is off); slots = num_sms * (max(h_p, 1) if limited else k);
+    n0 = number of base items.  If prefill_splits == 1, or n0 == 0, or
+    n0 >= slots: every item has S = 1 piece.  Otherwise W = sum of n over the
+    base items, tau = max(8, ceil(W / slots)) and an item of n tiles gets
+    S = min(smax, max(1, floor(n / tau))) pieces, smax = prefill_splits if
+    >= 2 else 16.  Piece s covers key tiles [floor(s n / S), floor((s+1) n / S)),
+    i.e. keys [64 j0, min(64 j1, kv_end)); every piece is at least 8 tiles
+    long, so every row of the tile sees at least one key of every piece.
+    Prefill items (q0, h, kv_end, request, j0, j1, partial, merge): partial =
+    running index over the pieces of split items in base-item order, else
+    -1; merge = index of the item's prefill merge entry, else -1.  Prefill
+    merge entries (first partial, S, 0, 0), one per split base item, in
+    base-item order.  All pieces are then stably sorted by their key count,
+    longest first.
   Decode split: W = num_sms * ctas_per_sm * decode warps per CTA (6, or 4 in
     the four-warp ablation); cap = max_waves * W;
     pages_r = ceil(L_r / 16); N = Hkv * sum pages_r; maxp = max pages_r;
@@ -61,6 +81,10 @@ import numpy as np
 
 PAGE = 16
 BM = 128
+BN = 64                     # keys per prefill key tile
+SPLIT_LIMIT_TOKENS = 1536   # prefill tokens up to which the split leaves room for co-located decode CTAs
+MIN_SPLIT_TILES = 8         # shortest prefill piece, in key tiles
+MAX_PREFILL_SPLITS = 16
 DECODE_WARPS = 6            # per CTA: every warp decodes (4 in the four-warp ablation)
 COST_RATIO = 248
 MAX_SMS = 512
@@ -75,7 +99,7 @@ class PlanError(ValueError):
 
 @dataclasses.dataclass
 class PlanRef:
-    prefill_items: np.ndarray   # int32 [n, 4]: q0, q head, kv_end, request
+    prefill_items: np.ndarray   # int32 [n, 8]: q0, q head, kv_end, request, j0, j1, partial, merge
     decode_items: np.ndarray    # int32 [n, 8]
     merge_items: np.ndarray     # int32 [n, 4]
     ctas_per_sm: int
@@ -84,6 +108,8 @@ class PlanRef:
     chunk_pages: int
     num_partials: int
     prefill_requests: np.ndarray = None   # int32 [NP, 4]: q_start, P, C, 0
+    prefill_merge_items: np.ndarray = None   # int32 [n, 4]: first partial, pieces, 0, 0
+    num_prefill_partials: int = 0
 
 
 def _ceil(a: int, b: int) -> int:
@@ -100,7 +126,8 @@ def plan_ref(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
 def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms: int,
                      prefill_qo_lens: Sequence[int], prefill_kv_lens: Sequence[int], decode_lens: Sequence[int], *,
                      page_size: int = 16, ctas_per_sm: int = 0, ratio_p: int = 0, ratio_d: int = 0,
-                     max_waves: int = 0, min_chunk_pages: int = 0, decode_warps: int = DECODE_WARPS) -> PlanRef:
+                     max_waves: int = 0, min_chunk_pages: int = 0, decode_warps: int = DECODE_WARPS,
+                     prefill_splits: int = 0, split_unlimited: bool = False) -> PlanRef:
     """NP prefill requests (block-table rows 0..NP-1) and B decodes (rows NP..NP+B-1)."""
     Hq, Hkv, d = int(num_q_heads), int(num_kv_heads), int(head_dim)
     pre_qo = [int(x) for x in prefill_qo_lens]
@@ -114,7 +141,7 @@ def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms
         raise PlanError("unsupported")
     if not (1 <= num_sms <= MAX_SMS) or ctas_per_sm not in (0, 1, 2):
         raise PlanError("invalid launch knobs")
-    if ratio_p < 0 or ratio_d < 0 or max_waves < 0 or min_chunk_pages < 0:
+    if ratio_p < 0 or ratio_d < 0 or max_waves < 0 or min_chunk_pages < 0 or not (0 <= prefill_splits <= MAX_PREFILL_SPLITS):
         raise PlanError("invalid knobs")
     if len(pre_qo) != len(pre_kv) or len(pre_qo) > MAX_PREFILL_REQUESTS:
         raise PlanError("invalid prefill requests")
@@ -142,7 +169,6 @@ def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms
         for t in range(_ceil(P, BM) - 1, -1, -1):
             for h in range(Hq):
                 pre.append((BM * t, h, C + min(BM * (t + 1), P), i))
-    pre.sort(key=lambda e: -e[2])          # stable: equal kv_end keep (request, tile, head) order
     preq, q_start = [], 0
     for P, C in zip(pre_qo, ctx):
         preq.append((q_start, P, C, 0))
@@ -217,8 +243,36 @@ def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms
             gg = math.gcd(p_, d_)
             p_, d_ = p_ // gg, d_ // gg
 
+    # prefill KV split
+    h_p = sum(1 for t in range(k) if (p_ + d_) > 0 and t % (p_ + d_) < p_)
+    limited = B > 0 and sum(pre_qo) <= SPLIT_LIMIT_TOKENS and not split_unlimited
+    slots = num_sms * (max(h_p, 1) if limited else k)
+    tiles = [_ceil(kv_end, BN) for (_, _, kv_end, _) in pre]
+    n0 = len(pre)
+    if prefill_splits == 1 or n0 == 0 or n0 >= slots:
+        nsplit = [1] * n0
+    else:
+        tau = max(MIN_SPLIT_TILES, _ceil(sum(tiles), slots))
+        smax = prefill_splits if prefill_splits >= 2 else MAX_PREFILL_SPLITS
+        nsplit = [min(smax, max(1, n // tau)) for n in tiles]
+    pieces, pmerge, nppart = [], [], 0
+    for (q0, h, kv_end, i), n, S in zip(pre, tiles, nsplit):
+        midx = len(pmerge) if S > 1 else -1
+        if S > 1:
+            pmerge.append((nppart, S, 0, 0))
+        for sp in range(S):
+            j0, j1 = (sp * n) // S, ((sp + 1) * n) // S
+            part = -1
+            if S > 1:
+                part = nppart
+                nppart += 1
+            pieces.append((q0, h, kv_end, i, j0, j1, part, midx))
+    # longest piece first; stable, so equal lengths keep (request, tile, head, piece) order
+    pieces.sort(key=lambda e: -(min(BN * e[5], e[2]) - BN * e[4]))
+
     def arr(rows, w):
         a = np.asarray(rows, dtype=np.int32)
         return a.reshape(len(rows), w)
 
-    return PlanRef(arr(pre, 4), arr([e[4] for e in dec], 8), arr(merge, 4), k, p_, d_, c, npart, arr(preq, 4))
+    return PlanRef(arr(pieces, 8), arr([e[4] for e in dec], 8), arr(merge, 4), k, p_, d_, c, npart, arr(preq, 4),
+                   arr(pmerge, 4), nppart)

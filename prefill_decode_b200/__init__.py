@@ -32,19 +32,22 @@ POD_FLAG_SELFTEST_TIMEOUT = 8
 POD_FLAG_TWO_STREAMS = 16
 POD_FLAG_SM_PARTITION = 32
 POD_FLAG_DECODE_FOUR_WARPS = 64
+POD_FLAG_PREFILL_SPLIT_UNLIMITED = 128
 
 EXPORTED = [
     "pod_attn_plan", "pod_attn_plan_get_info", "pod_attn_plan_tables", "pod_attn_upload", "pod_attn_run",
     "pod_attn_plan_set_events", "pod_attn_event_create", "pod_attn_event_destroy", "pod_attn_event_elapsed_ms",
     "pod_attn_plan_destroy", "pod_attn_status_string", "pod_attn_last_cuda_error", "pod_attn_run_static",
-    "pod_attn_plan_batched", "pod_attn_plan_prefill_requests",
+    "pod_attn_plan_batched", "pod_attn_plan_prefill_requests", "pod_attn_plan_prefill_merges",
+    "pod_attn_run_fp8kv",
 ]
 
 
 class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_sms", "ctas_per_sm",
-        "ratio_prefill", "ratio_decode", "max_waves", "min_chunk_pages")] + [("flags", ctypes.c_uint32)]
+        "ratio_prefill", "ratio_decode", "max_waves", "min_chunk_pages", "max_prefill_splits")] + [
+            ("flags", ctypes.c_uint32)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -52,7 +55,8 @@ class PlanInfo(ctypes.Structure):
         "num_prefill_items", "num_decode_items", "num_merge_items", "num_partials", "ctas_per_sm",
         "ratio_prefill", "ratio_decode", "chunk_pages", "num_sms", "grid")] + [(n, ctypes.c_int64) for n in (
             "workspace_bytes", "error_offset", "prefill_flops", "decode_flops", "kv_bytes", "qo_bytes", "table_bytes")] + [
-            (n, ctypes.c_int32) for n in ("num_prefill_requests", "num_prefill_rows")]
+            (n, ctypes.c_int32) for n in ("num_prefill_requests", "num_prefill_rows", "num_prefill_partials",
+                                          "num_prefill_merge_items")] + [("rescale_count_offset", ctypes.c_int64)]
 
 
 class PodError(RuntimeError):
@@ -78,6 +82,7 @@ def lib() -> ctypes.CDLL:
         L.pod_attn_plan_batched.argtypes = [ctypes.POINTER(Config), i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
                                             i32, ctypes.POINTER(i32), ctypes.POINTER(vp), ctypes.POINTER(sz)]
         L.pod_attn_plan_prefill_requests.argtypes = [vp, vp]
+        L.pod_attn_plan_prefill_merges.argtypes = [vp, vp]
         L.pod_attn_plan_get_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
         L.pod_attn_plan_tables.argtypes = [vp, vp, vp, vp]
         L.pod_attn_upload.argtypes = [vp, vp, sz, vp]
@@ -92,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.pod_attn_status_string.restype = ctypes.c_char_p
         L.pod_attn_last_cuda_error.argtypes = []
         L.pod_attn_run_static.argtypes = [vp, vp, vp, vp, vp, i64, vp, i32, vp, ctypes.c_float, vp, vp, vp]
+        L.pod_attn_run_fp8kv.argtypes = [vp, vp, vp, vp, vp, i64, vp, vp, i64, vp, vp, vp, i32, vp, ctypes.c_float,
+                                         vp, vp, vp, sz, vp, vp]
         for n in EXPORTED:
             if n not in ("pod_attn_plan_destroy", "pod_attn_status_string"):
                 getattr(L, n).restype = ctypes.c_int
@@ -135,10 +142,10 @@ class Plan:
     def __init__(self, num_q_heads: int, num_kv_heads: int, head_dim: int, prefill_len,
                  prefill_kv_len, decode_lens: Sequence[int], *, num_sms: int = 0,
                  ctas_per_sm: int = 0, ratio: Tuple[int, int] = (0, 0), max_waves: int = 0,
-                 min_chunk_pages: int = 0, flags: int = 0, page_size: int = 16):
+                 min_chunk_pages: int = 0, max_prefill_splits: int = 0, flags: int = 0, page_size: int = 16):
         L = lib()
         self.cfg = Config(num_q_heads, num_kv_heads, head_dim, page_size, num_sms, ctas_per_sm,
-                          ratio[0], ratio[1], max_waves, min_chunk_pages, flags)
+                          ratio[0], ratio[1], max_waves, min_chunk_pages, max_prefill_splits, flags)
         lens = np.ascontiguousarray(np.asarray(decode_lens, dtype=np.int32))
         self._lens = lens
         h = ctypes.c_void_p()
@@ -178,9 +185,16 @@ class Plan:
         _check(lib().pod_attn_plan_prefill_requests(self._h, out.ctypes.data), "pod_attn_plan_prefill_requests")
         return out
 
+    def prefill_merges(self) -> np.ndarray:
+        """int32 [num_prefill_merge_items, 4]: first partial, pieces, 0, 0."""
+        out = np.zeros((self.info.num_prefill_merge_items, 4), dtype=np.int32)
+        _check(lib().pod_attn_plan_prefill_merges(self._h, out.ctypes.data), "pod_attn_plan_prefill_merges")
+        return out
+
     def tables(self):
+        """Host copies of the prefill items [n, 8], decode items [n, 8] and decode merge items [n, 4]."""
         i = self.info
-        pre = np.zeros((i.num_prefill_items, 4), dtype=np.int32)
+        pre = np.zeros((i.num_prefill_items, 8), dtype=np.int32)
         dec = np.zeros((i.num_decode_items, 8), dtype=np.int32)
         mer = np.zeros((i.num_merge_items, 4), dtype=np.int32)
         _check(lib().pod_attn_plan_tables(self._h, pre.ctypes.data, dec.ctypes.data, mer.ctypes.data),
@@ -201,6 +215,22 @@ class Plan:
                                   int(num_blocks), _ptr(block_table), int(block_table_stride), _ptr(kv_lens),
                                   float(scale), _ptr(o_prefill), _ptr(o_decode), _ptr(workspace),
                                   int(workspace_bytes), _ptr(trace), _stream(stream)), "pod_attn_run")
+
+    def run_fp8kv(self, q_prefill, q_decode, k_cache, v_cache, num_blocks: int, k_cache_fp8, v_cache_fp8,
+                  num_blocks_fp8: int, k_scale, v_scale, block_table, block_table_stride: int, kv_lens,
+                  scale: float, o_prefill, o_decode, workspace, trace=None, stream=None,
+                  workspace_bytes: Optional[int] = None) -> None:
+        """pod_attn_run_fp8kv: the decode requests read the e4m3 pools (uint8) with per-kv-head fp32
+        scales; the prefill requests read the bf16 pools."""
+        if workspace_bytes is None:
+            workspace_bytes = (workspace.numel() * workspace.element_size()
+                               if hasattr(workspace, "numel") else self.workspace_bytes)
+        _check(lib().pod_attn_run_fp8kv(self._h, _ptr(q_prefill), _ptr(q_decode), _ptr(k_cache), _ptr(v_cache),
+                                        int(num_blocks), _ptr(k_cache_fp8), _ptr(v_cache_fp8), int(num_blocks_fp8),
+                                        _ptr(k_scale), _ptr(v_scale), _ptr(block_table), int(block_table_stride),
+                                        _ptr(kv_lens), float(scale), _ptr(o_prefill), _ptr(o_decode),
+                                        _ptr(workspace), int(workspace_bytes), _ptr(trace), _stream(stream)),
+               "pod_attn_run_fp8kv")
 
     def set_events(self, ev_start: Optional[int], ev_stop: Optional[int]) -> None:
         _check(lib().pod_attn_plan_set_events(self._h, ev_start, ev_stop), "pod_attn_plan_set_events")

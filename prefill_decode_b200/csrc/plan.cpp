@@ -3,10 +3,11 @@
 //
 // The knobs come from the POD-Attention explainer ("How POD-Attention overlaps
 // prefill and decode"): CTAs per SM, split-KV capped at two waves, CTAs
-// allocated in proportion to the prefill:decode mix.  The pages give no
-// formula, so the rule here is this library's own, written out in prose in
-// oracle/plan_ref.py's docstring (the test oracle restates it in Python and the
-// tests compare the two bit for bit).  Integer arithmetic only.
+// allocated in proportion to the prefill:decode mix; the prefill's KV split
+// leaves room for co-located decode CTAs while the prefill is short (FlashInfer
+// PR "Limit kv split when prefill tokens <= 1536").  The pages give no formula,
+// so the rule is this library's own; it is written out in include/pod_attn.h
+// (above pod_attn_plan).  Integer arithmetic only.
 #include <algorithm>
 #include <cstring>
 #include <new>
@@ -19,6 +20,8 @@ namespace {
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 constexpr int kMaxHeads = 4096;   // query heads per plan
+constexpr int32_t kSplitLimitTokens = 1536;   // prefill tokens up to which the split counts co-located decode CTAs
+constexpr int32_t kMinSplitTiles = 8;         // shortest prefill piece, in 64-key tiles
 constexpr int kDecodeWarpsAll = 6;  // decode warps per CTA when every warp decodes (the kernel's 192 threads)
 
 struct DecEntry {
@@ -38,7 +41,8 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
   if (g > 8 || (d != 64 && d != 128) || cfg->page_size != kPage) return POD_ERR_UNSUPPORTED;
   if (num_sms < 1 || num_sms > kMaxSms) return POD_ERR_INVALID_ARG;
   if (cfg->ctas_per_sm < 0 || cfg->ctas_per_sm > 2) return POD_ERR_INVALID_ARG;
-  if (cfg->ratio_prefill < 0 || cfg->ratio_decode < 0 || cfg->max_waves < 0 || cfg->min_chunk_pages < 0)
+  if (cfg->ratio_prefill < 0 || cfg->ratio_decode < 0 || cfg->max_waves < 0 || cfg->min_chunk_pages < 0 ||
+      cfg->max_prefill_splits < 0 || cfg->max_prefill_splits > kMaxPrefillPieces)
     return POD_ERR_INVALID_ARG;
   if (NP < 0 || NP > kMaxPrefillRequests || (NP > 0 && (!pre_qo || !pre_kv))) return POD_ERR_INVALID_ARG;
   int64_t sumP = 0;
@@ -91,21 +95,17 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
   pl->grid = num_sms * k;
   pl->decode_lens.assign(lens, lens + B);
 
-  // ---- prefill items: one 128-row query tile of one query head, per request last
-  // tile first, then all requests' items longest (largest kv_end) first, stably
-  struct PreEntry {
-    int32_t item[kPrefillItemInts];
+  // ---- base prefill items: one 128-row query tile of one query head, per request last
+  // tile first (they are cut into KV pieces and ordered once the ratio is known)
+  struct BaseItem {
+    int32_t q0, h, kv_end, req;
   };
-  std::vector<PreEntry> pents;
+  std::vector<BaseItem> base;
   for (int32_t i = 0; i < NP; ++i) {
     const int32_t P = pre_qo[i], C = ctx[i];
     for (int32_t t = (int32_t)ceil_div(P, kBM) - 1; t >= 0; --t)
-      for (int32_t h = 0; h < Hq; ++h) pents.push_back(PreEntry{{kBM * t, h, C + std::min(kBM * (t + 1), P), i}});
+      for (int32_t h = 0; h < Hq; ++h) base.push_back(BaseItem{kBM * t, h, C + std::min(kBM * (t + 1), P), i});
   }
-  std::stable_sort(pents.begin(), pents.end(),
-                   [](const PreEntry& a, const PreEntry& b) { return a.item[2] > b.item[2]; });
-  for (const PreEntry& e : pents) pl->pre.insert(pl->pre.end(), e.item, e.item + kPrefillItemInts);
-  pl->n_pre = (int32_t)pents.size();
   int32_t q_start = 0;
   for (int32_t i = 0; i < NP; ++i) {
     const int32_t rq[kPrefillReqInts] = {q_start, pre_qo[i], ctx[i], 0};
@@ -185,7 +185,7 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
       rp = cfg->ratio_prefill / gg;
       rd = cfg->ratio_decode / gg;
     }
-  } else if (pl->n_pre == 0) {
+  } else if (base.empty()) {
     rp = 0; rd = 1;
   } else if (pl->n_dec == 0) {
     rp = 1; rd = 0;
@@ -210,24 +210,75 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
   pl->ratio_p = rp;
   pl->ratio_d = rd;
 
+  // ---- prefill KV split: fill the prefill CTA slots when the base items leave some empty;
+  // a short prefill (<= 1536 tokens) next to decode work counts only its prefill-home CTAs
+  {
+    int32_t hp = 0;
+    for (int32_t t = 0; t < k; ++t)
+      if (rp + rd > 0 && t % (rp + rd) < rp) ++hp;
+    const bool limited = B > 0 && sumP <= kSplitLimitTokens && !(cfg->flags & POD_FLAG_PREFILL_SPLIT_UNLIMITED);
+    const int64_t slots = (int64_t)num_sms * (limited ? std::max<int32_t>(hp, 1) : k);
+    const int64_t n0 = (int64_t)base.size();
+    std::vector<int32_t> nsplit(base.size(), 1);
+    if (cfg->max_prefill_splits != 1 && n0 > 0 && n0 < slots) {
+      int64_t tiles = 0;
+      for (const BaseItem& b : base) tiles += ceil_div(b.kv_end, kBN);
+      const int64_t tau = std::max<int64_t>(kMinSplitTiles, ceil_div(tiles, slots));
+      const int32_t smax = cfg->max_prefill_splits >= 2 ? cfg->max_prefill_splits : kMaxPrefillPieces;
+      for (size_t i = 0; i < base.size(); ++i)
+        nsplit[i] = (int32_t)std::min<int64_t>(smax, std::max<int64_t>(1, ceil_div(base[i].kv_end, kBN) / tau));
+    }
+    struct PreEntry {
+      int32_t keys;
+      int32_t item[kPrefillItemInts];
+    };
+    std::vector<PreEntry> pents;
+    int32_t nppart = 0;
+    for (size_t i = 0; i < base.size(); ++i) {
+      const BaseItem& b = base[i];
+      const int32_t n = (int32_t)ceil_div(b.kv_end, kBN), S = nsplit[i];
+      const int32_t midx = S > 1 ? (int32_t)(pl->pmerge.size() / kPrefillMergeInts) : -1;
+      if (S > 1) {
+        const int32_t m[kPrefillMergeInts] = {nppart, S, 0, 0};
+        pl->pmerge.insert(pl->pmerge.end(), m, m + kPrefillMergeInts);
+      }
+      for (int32_t sp = 0; sp < S; ++sp) {
+        const int32_t j0 = (int32_t)(((int64_t)sp * n) / S), j1 = (int32_t)(((int64_t)(sp + 1) * n) / S);
+        const int32_t part = S > 1 ? nppart++ : -1;
+        pents.push_back(PreEntry{std::min(kBN * j1, b.kv_end) - kBN * j0,
+                                 {b.q0, b.h, b.kv_end, b.req, j0, j1, part, midx}});
+      }
+    }
+    // longest piece first; stable, so equal lengths keep (request, tile, head, piece) order
+    std::stable_sort(pents.begin(), pents.end(), [](const PreEntry& a, const PreEntry& b) { return a.keys > b.keys; });
+    for (const PreEntry& e : pents) pl->pre.insert(pl->pre.end(), e.item, e.item + kPrefillItemInts);
+    pl->n_pre = (int32_t)pents.size();
+    pl->n_ppart = nppart;
+    pl->n_pmerge = (int32_t)(pl->pmerge.size() / kPrefillMergeInts);
+  }
+
   // ---- workspace layout and the host image of the tables
   pl->off_merge_cnt = kCountersBytes;
-  pl->off_pre = align_up(pl->off_merge_cnt + 4LL * pl->n_merge, 256);
+  pl->off_pmerge_cnt = pl->off_merge_cnt + 4LL * pl->n_merge;
+  pl->off_pre = align_up(pl->off_pmerge_cnt + 4LL * kWarpsPerCta * pl->n_pmerge, 256);
   pl->off_dec = align_up(pl->off_pre + 4LL * kPrefillItemInts * pl->n_pre, 256);
   pl->off_merge = align_up(pl->off_dec + 4LL * kDecodeItemInts * pl->n_dec, 256);
   pl->off_preq = align_up(pl->off_merge + 4LL * kMergeItemInts * pl->n_merge, 256);
-  pl->off_part_o = align_up(pl->off_preq + 4LL * kPrefillReqInts * NP, 256);
+  pl->off_pmerge = align_up(pl->off_preq + 4LL * kPrefillReqInts * NP, 256);
+  pl->off_part_o = align_up(pl->off_pmerge + 4LL * kPrefillMergeInts * pl->n_pmerge, 256);
   pl->off_part_lse = align_up(pl->off_part_o + 4LL * g * d * npart, 256);
-  pl->ws_bytes = align_up(pl->off_part_lse + 4LL * g * npart, 256);
+  pl->off_ppart_o = align_up(pl->off_part_lse + 4LL * g * npart, 256);
+  pl->off_ppart_lse = align_up(pl->off_ppart_o + 4LL * kBM * d * pl->n_ppart, 256);
+  pl->ws_bytes = align_up(pl->off_ppart_lse + 4LL * kBM * pl->n_ppart, 256);
   pl->image.assign((size_t)(pl->off_part_o - kCountersBytes), 0);
-  if (!pl->pre.empty())
-    std::memcpy(pl->image.data() + (pl->off_pre - kCountersBytes), pl->pre.data(), pl->pre.size() * 4);
-  if (!pl->dec.empty())
-    std::memcpy(pl->image.data() + (pl->off_dec - kCountersBytes), pl->dec.data(), pl->dec.size() * 4);
-  if (!pl->merge.empty())
-    std::memcpy(pl->image.data() + (pl->off_merge - kCountersBytes), pl->merge.data(), pl->merge.size() * 4);
-  if (!pl->preq.empty())
-    std::memcpy(pl->image.data() + (pl->off_preq - kCountersBytes), pl->preq.data(), pl->preq.size() * 4);
+  auto put = [&](int64_t off, const std::vector<int32_t>& v) {
+    if (!v.empty()) std::memcpy(pl->image.data() + (off - kCountersBytes), v.data(), v.size() * 4);
+  };
+  put(pl->off_pre, pl->pre);
+  put(pl->off_dec, pl->dec);
+  put(pl->off_merge, pl->merge);
+  put(pl->off_preq, pl->preq);
+  put(pl->off_pmerge, pl->pmerge);
   *out = pl;
   return POD_OK;
 }

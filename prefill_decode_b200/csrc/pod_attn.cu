@@ -47,6 +47,8 @@ struct alignas(64) PodParams {
   CUtensorMap tm_k;    // K cache viewed as 2D [num_blocks*Hkv*16 rows, d], box {64, 16}, 128B swizzle
   CUtensorMap tm_kp;   // K cache as 3D [d/64 halves][rows][64]: one box {64, 16, d/64} = one whole page
   CUtensorMap tm_vp;   // V cache, same view
+  CUtensorMap tm_k8;   // e4m3 K cache of the decode requests, 2D [rows, d] bytes, box {d, 16} (unused for bf16)
+  CUtensorMap tm_v8;   // e4m3 V cache, same view
   const __nv_bfloat16* q_pre;
   const __nv_bfloat16* q_dec;
   __nv_bfloat16* o_pre;
@@ -54,17 +56,23 @@ struct alignas(64) PodParams {
   const int32_t* block_table;
   const int32_t* kv_lens;
   int32_t* counters;
-  const int4* pre_items;
+  const int4* pre_items;   // two int4 per item: q0, q head, kv_end, request | j0, j1, partial, merge
   const int4* dec_items;   // two int4 per item
   const int4* merge_items; // r, kvh, first_partial, num_splits
   const int4* pre_reqs;    // per prefill request: first row in q_pre / o_pre, P, C, 0
-  int32_t* merge_cnt;      // splits finished per merge item (zero at launch)
+  const int4* pmerge_items; // per split prefill item: first partial, pieces, 0, 0
+  int32_t* merge_cnt;      // splits finished per decode merge item (zero at launch)
+  int32_t* pmerge_cnt;     // pieces finished per split prefill item and softmax warp (zero at launch)
   float* part_o;
   float* part_lse;
+  float* ppart_o;          // prefill piece partials: O [n, 128, d] (normalised) and LSE [n, 128], log2 domain
+  float* ppart_lse;
   int32_t* trace;
   int32_t bt_stride;
   int32_t kv_rows;         // num_blocks * Hkv * 16 (rows of the K/V tensor maps)
   int32_t num_blocks;
+  int32_t kv_rows8;        // the same for the e4m3 cache of the decode requests
+  int32_t num_blocks8;
   int32_t n_pre, n_dec;
   int32_t Hq, Hkv, g, NP, B;   // NP prefill requests own block-table rows 0..NP-1
   int32_t ratio_p, ratio_d;
@@ -75,6 +83,8 @@ struct alignas(64) PodParams {
   int32_t partition_sms;   // > 0: roles by SM id instead of per-SM tickets (ablation)
   int32_t decode_warps;    // warps of a CTA that run decode items: 4, or 6 (the MMA and TMA warps too)
   float scale_log2;        // softmax scale * log2(e)
+  const float* k_scale8;   // e4m3 caches: per kv head, dequantised value = scale * stored value
+  const float* v_scale8;
 };
 
 constexpr int kThreads = 192;        // warps 0-3: softmax (prefill) / decode units; warp 4: MMA; warp 5: TMA
@@ -123,9 +133,14 @@ struct Cfg {
   static constexpr int kDecStage = 2 * kPageBytes;            // K page + V page
   static constexpr int kNS = (kPrefillSmem / kWarpsPerCta) / kDecStage;   // decode ring depth per warp
   static constexpr int kNSAll = (kPrefillSmem / kAllWarps) / kDecStage;    // ... when all warps decode
+  static constexpr int kPageBytes8 = kPage * D;               // the same page in e4m3
+  static constexpr int kDecStage8 = 2 * kPageBytes8;
+  static constexpr int kNS8 = (kPrefillSmem / kWarpsPerCta) / kDecStage8;
+  static constexpr int kNSAll8 = (kPrefillSmem / kAllWarps) / kDecStage8;
   static constexpr int kSmem = kPrefillSmem;
-  static constexpr int kNumBars =
-      kBarDecode + (kWarpsPerCta * kNS > kAllWarps * kNSAll ? kWarpsPerCta * kNS : kAllWarps * kNSAll);
+  static constexpr int cmax(int a, int b) { return a > b ? a : b; }
+  static constexpr int kNumBars = kBarDecode + cmax(cmax(kWarpsPerCta * kNS, kAllWarps * kNSAll),
+                                                    cmax(kWarpsPerCta * kNS8, kAllWarps * kNSAll8));
   static constexpr int kCtrlBytes = 512;                      // barriers, TMEM address, broadcast slots
   static_assert((kNumBars + 1) * 8 + 32 <= kCtrlBytes, "control block too small");   // + the self-test barrier
   // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) can share an SM
@@ -136,6 +151,10 @@ static_assert(Cfg<128>::kNSAll >= 2 && Cfg<64>::kNSAll >= 2, "decode ring too sh
 static_assert(kAllWarps * Cfg<128>::kNSAll * Cfg<128>::kDecStage <= Cfg<128>::kPrefillSmem &&
                   kAllWarps * Cfg<64>::kNSAll * Cfg<64>::kDecStage <= Cfg<64>::kPrefillSmem,
               "decode rings exceed the shared-memory union");
+static_assert(kAllWarps * Cfg<128>::kNSAll8 * Cfg<128>::kDecStage8 <= Cfg<128>::kPrefillSmem &&
+                  kWarpsPerCta * Cfg<64>::kNS8 * Cfg<64>::kDecStage8 <= Cfg<64>::kPrefillSmem &&
+                  Cfg<128>::kDecStage8 % 1024 == 0,
+              "e4m3 decode rings exceed the shared-memory union or break the swizzle alignment");
 
 __device__ __forceinline__ void record_error(const PodParams& p, int code, int info) {
   if (atomicCAS(&p.counters[kErrorWord], 0, code) == 0) atomicExch(&p.counters[kErrorInfo], info);
@@ -147,6 +166,14 @@ __device__ __forceinline__ int kv_row(const PodParams& p, int blk, int kvh) {
   if (blk < 0 || blk >= p.num_blocks) {
     record_error(p, POD_ERR_BOUNDS, blk);
     return p.kv_rows;
+  }
+  return (blk * p.Hkv + kvh) * kPage;
+}
+// ... of the e4m3 cache (decode requests of pod_attn_run_fp8kv)
+__device__ __forceinline__ int kv_row8(const PodParams& p, int blk, int kvh) {
+  if (blk < 0 || blk >= p.num_blocks8) {
+    record_error(p, POD_ERR_BOUNDS, blk);
+    return p.kv_rows8;
   }
   return (blk * p.Hkv + kvh) * kPage;
 }
@@ -162,6 +189,20 @@ struct PrefillSmem {
   __device__ uint8_t* v(uint32_t t) const { return base + Cfg<D>::kOffV + (t % Cfg<D>::kVSlots) * Cfg<D>::kKTile; }
   __device__ uint8_t* pbuf(uint32_t t) const { return base + Cfg<D>::kOffP + (t & 1u) * Cfg<D>::kPBytes; }
 };
+
+// One prefill work item: query rows q0 .. q0+127 of `req` for query head qh,
+// key tiles j0 .. j1-1 (64 keys each, absolute within the request) of a causal
+// range that ends at kv_end.  part < 0: the item covers every key tile and
+// writes bf16 O; otherwise it is one KV piece of a split item and writes a
+// partial, and the last piece to finish merges them (prefill merge item midx).
+struct PreItem {
+  int q0, qh, kv_end, req, j0, j1, part, midx;
+};
+
+__device__ __forceinline__ PreItem load_pre_item(const PodParams& p, int i) {
+  const int4 a = __ldg(&p.pre_items[2 * i]), b = __ldg(&p.pre_items[2 * i + 1]);
+  return PreItem{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+}
 
 // Block ids of the prefill request's pages, read 32 at a time (one per lane) a
 // window ahead of use: `cur` holds pages [32 w, 32 w + 32) (key tiles 8w ..
@@ -221,34 +262,36 @@ __device__ __forceinline__ void issue_vtile(const PodParams& p, uint8_t* dst, ui
 // TMA warp of one prefill item: K into a 3-deep ring and V into a 2-deep
 // ring; K_{t+3} goes into slot t%3 once S_t finished, V_{t+2} into slot t&1
 // once P.V_t finished.  `t0` = key tiles this CTA processed before this item
-// (it indexes every ring and mbarrier phase).
+// (it indexes every ring and mbarrier phase); the item's tiles are j0 .. j1-1.
 template <int D>
-__device__ bool prefill_tma(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t t0) {
+__device__ bool prefill_tma(const PodParams& p, const PreItem& it, uint8_t* smem, uint64_t* bars, uint32_t t0) {
   using CF = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  const int qh = it.y, kv_end = it.z, req = it.w;
-  const int kvh = qh / p.g;
-  const int nkb = (kv_end + kBN - 1) / kBN;
+  const int kv_end = it.kv_end, j0 = it.j0;
+  const int kvh = it.qh / p.g;
+  const int nkb = it.j1 - it.j0;
   const PrefillSmem<D> sm{smem};
-  const int* bt_row = p.block_table + (size_t)req * p.bt_stride;
-  if (lane == 0 && p.kv_lens && __ldg(&p.kv_lens[req]) < kv_end) record_error(p, POD_ERR_PLAN_MISMATCH, req);
-  PageWindows pw{load_page_window(p, bt_row, 0, kv_end, lane), load_page_window(p, bt_row, 1, kv_end, lane), 0};
+  const int* bt_row = p.block_table + (size_t)it.req * p.bt_stride;
+  if (lane == 0 && p.kv_lens && __ldg(&p.kv_lens[it.req]) < kv_end) record_error(p, POD_ERR_PLAN_MISMATCH, it.req);
+  const int w0 = j0 >> 3;   // 32-page windows hold 8 key tiles
+  PageWindows pw{load_page_window(p, bt_row, w0, kv_end, lane), load_page_window(p, bt_row, w0 + 1, kv_end, lane),
+                 w0};
   for (int j = 0; j < nkb && j < CF::kKSlots; ++j) {
     const uint32_t t = t0 + j;
-    const int r = tile_page_row(p, pw, j, kvh, kv_end, lane);
+    const int r = tile_page_row(p, pw, j0 + j, kvh, kv_end, lane);
     issue_tile<D>(&p.tm_k, sm.k(t), &bars[kBarKFull + t % 3], r, lane);
     if (j < CF::kVSlots) issue_vtile<D>(p, sm.v(t), &bars[kBarVFull + (t & 1u)], r, lane);
   }
   for (int j = 0; j + CF::kVSlots < nkb; ++j) {
     const uint32_t t = t0 + j;
-    if (((j + CF::kVSlots) >> 3) > pw.w) {   // tile j+2 enters the next window; fetch the one after it
+    if (((j0 + j + CF::kVSlots) >> 3) > pw.w) {   // tile j+2 enters the next window; fetch the one after it
       ++pw.w;
       pw.cur = pw.nxt;
       pw.nxt = load_page_window(p, bt_row, pw.w + 1, kv_end, lane);
     }
     const bool more_k = j + CF::kKSlots < nkb;
-    const int rk = more_k ? tile_page_row(p, pw, j + CF::kKSlots, kvh, kv_end, lane) : 0;
-    const int rv = tile_page_row(p, pw, j + CF::kVSlots, kvh, kv_end, lane);
+    const int rk = more_k ? tile_page_row(p, pw, j0 + j + CF::kKSlots, kvh, kv_end, lane) : 0;
+    const int rv = tile_page_row(p, pw, j0 + j + CF::kVSlots, kvh, kv_end, lane);
     if (more_k) {                // K first: S_{t+3} is issued well before P.V_{t+2}
       if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKEmpty + t % 3], (t / 3) & 1u, kWaitLimitNs))) return false;
       issue_tile<D>(&p.tm_k, sm.k(t + CF::kKSlots), &bars[kBarKFull + t % 3], rk, lane);
@@ -265,12 +308,12 @@ __device__ bool prefill_tma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
 // Commits free the K slot right after S_t and the V slot and the P buffer
 // after P.V_t.
 template <int D>
-__device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t tmem, uint32_t t0,
-                            uint32_t nq) {
+__device__ bool prefill_mma(const PodParams& p, const PreItem& it, uint8_t* smem, uint64_t* bars, uint32_t tmem,
+                            uint32_t t0, uint32_t nq) {
   using CF = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  const int kv_end = it.z;
-  const int nkb = (kv_end + kBN - 1) / kBN;
+  const int kv_end = it.kv_end;
+  const int nkb = it.j1 - it.j0;
   const PrefillSmem<D> sm{smem};
   constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false, false);
   constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, false, true);
@@ -317,7 +360,7 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
     const bool wp = mbar_wait(&bars[kBarVFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs) &&
                     mbar_wait(&bars[kBarPFull + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs);
     if (!__all_sync(0xffffffffu, wp)) return false;
-    const int valid = kv_end - j * kBN;
+    const int valid = kv_end - (it.j0 + j) * kBN;
     if (valid < kBN) {           // V rows past the request's end may hold anything: zero them
       uint8_t* vt = sm.v(t);
       for (int i = lane; i < (kBN - valid) * CF::kHalves * 8; i += 32) {
@@ -351,15 +394,19 @@ __device__ bool prefill_mma(const PodParams& p, int4 it, uint8_t* smem, uint64_t
 // at once), mask (bottom-right causal), online softmax in the exp2 domain with
 // a lazily updated row max (O in TMEM is rescaled only when the max grows by
 // more than 2^8), write P_t as bf16 into shared-memory buffer t&1 in the
-// K-major 128B-swizzled layout; finally O / l -> bf16 -> global.
+// K-major 128B-swizzled layout.  Epilogue: O / l -> bf16 -> global, or, for
+// one KV piece of a split item, the piece's partial (O / l in fp32 and its
+// log-sum-exp) and then the log-sum-exp merge of all the item's pieces, done
+// for each warp's 32 rows by the warp that finishes those rows' last piece
+// (a completion counter per item and softmax warp: no warp waits on another).
 template <int D>
-__device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint64_t* bars, uint32_t tmem,
-                                uint32_t t0, uint32_t nq) {
+__device__ bool prefill_softmax(const PodParams& p, const PreItem& it, int item, uint8_t* smem, uint64_t* bars,
+                                uint32_t tmem, uint32_t t0, uint32_t nq) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q0 = it.x, qh = it.y, kv_end = it.z;
-  const int4 rq = __ldg(&p.pre_reqs[it.w]);       // first row in q_pre / o_pre, P, C
+  const int q0 = it.q0, qh = it.qh, kv_end = it.kv_end, j0 = it.j0;
+  const int4 rq = __ldg(&p.pre_reqs[it.req]);     // first row in q_pre / o_pre, P, C
   const int q_first = rq.x, P = rq.y, C = rq.z;
-  const int nkb = (kv_end + kBN - 1) / kBN;
+  const int nkb = it.j1 - it.j0;
   const int row = tid;
   const int row_limit = min(C + q0 + row + 1, kv_end);
   const int full_tiles = (C + q0 + 1) / kBN;     // tiles visible to every row of this item
@@ -388,8 +435,9 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
     if (lane == 0) mbar_arrive(&bars[kBarQ]);
   }
   float m = -INFINITY, l = 0.f;
-  for (int j = 0; j < nkb; ++j) {
-    const uint32_t t = t0 + j;
+  for (int jj = 0; jj < nkb; ++jj) {
+    const int j = j0 + jj;       // absolute key tile
+    const uint32_t t = t0 + jj;
     if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull], t & 1u, kWaitLimitNs))) return false;
     tc_fence_after();
     float s[kBN];
@@ -400,7 +448,7 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars[kBarSFree]);   // S_{t+1} may overwrite the buffer now
     // P.V of tile t-2 read P buffer t&1; tiles of an earlier item finished with it
-    bool pbuf_free = j < 2;
+    bool pbuf_free = jj < 2;
     float mx = -INFINITY;        // row max of the raw scores; m below is in scaled (log2) units
     if (j >= full_tiles) {
       const int lim = row_limit - j * kBN;
@@ -410,11 +458,12 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
 #pragma unroll
     for (int k = 0; k < kBN / 2; ++k) mx = fmax3(mx, s[2 * k], s[2 * k + 1]);
     mx *= sl2;
-    if (j == 0) {
-      m = mx;
+    if (jj == 0) {
+      m = mx;                    // every row sees at least one key of a piece's first tile
     } else {
       const bool need = mx > m + 8.f;
       if (__any_sync(0xffffffffu, need)) {
+        if (p.trace && lane == 0) atomicAdd(&p.counters[kRescaleCount], 1);
         // O holds the P.V sums of the earlier tiles: wait for the last one, then rescale
         const uint32_t tp = t - 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone + (tp & 1u)], (tp >> 1) & 1u, kWaitLimitNs)))
@@ -468,27 +517,98 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars[kBarPFull + (t & 1u)]);
   }
-  // epilogue: O / l -> bf16, one 2*D-byte row per thread
+  // epilogue: O / l, one row per thread
   if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarOFinal], nq & 1u, kWaitLimitNs))) return false;
   tc_fence_after();
   const int q = q0 + row;
   const float inv = 1.f / l;
+  __nv_bfloat16* orow = p.o_pre + ((size_t)(q_first + q) * p.Hq + qh) * D;
+  // the piece fields are read again here rather than kept live through the tile loop
+  const int4 piece = ld_nc_v4(&p.pre_items[2 * item + 1]);   // j0, j1, partial, merge
+  const int part = piece.z, midx = piece.w;
+  if (part < 0) {
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      tmem_ld32(tmem + t_lane + kTmemO + c * 32, o);
+      tmem_wait_ld();
+      if (q < P) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint4 v;
+          v.x = pack_bf16(o[k * 8 + 0] * inv, o[k * 8 + 1] * inv);
+          v.y = pack_bf16(o[k * 8 + 2] * inv, o[k * 8 + 3] * inv);
+          v.z = pack_bf16(o[k * 8 + 4] * inv, o[k * 8 + 5] * inv);
+          v.w = pack_bf16(o[k * 8 + 6] * inv, o[k * 8 + 7] * inv);
+          dst[k] = v;
+        }
+      }
+    }
+    return true;
+  }
+  // one KV piece of a split item: write this piece's partial row
+  float* prow_o = p.ppart_o + ((size_t)part * kBM + row) * D;
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
     float o[32];
     tmem_ld32(tmem + t_lane + kTmemO + c * 32, o);
     tmem_wait_ld();
     if (q < P) {
-      uint4* dst = reinterpret_cast<uint4*>(p.o_pre + ((size_t)(q_first + q) * p.Hq + qh) * D + c * 32);
+      float4* dst = reinterpret_cast<float4*>(prow_o + c * 32);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint4 v;
-        v.x = pack_bf16(o[k * 8 + 0] * inv, o[k * 8 + 1] * inv);
-        v.y = pack_bf16(o[k * 8 + 2] * inv, o[k * 8 + 3] * inv);
-        v.z = pack_bf16(o[k * 8 + 4] * inv, o[k * 8 + 5] * inv);
-        v.w = pack_bf16(o[k * 8 + 6] * inv, o[k * 8 + 7] * inv);
-        dst[k] = v;
+      for (int k = 0; k < 8; ++k)
+        dst[k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv, o[4 * k + 3] * inv);
+    }
+  }
+  if (q < P) p.ppart_lse[(size_t)part * kBM + row] = m + __log2f(l);
+  // the warp that finishes its rows' last piece merges them (no waiting on other warps or CTAs)
+  const int4 pm = __ldg(&p.pmerge_items[midx]);   // first partial, pieces
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) last = atomicAdd(&p.pmerge_cnt[kWarpsPerCta * midx + warp], 1) == pm.y - 1;
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last || q >= P) return true;
+  __threadfence();
+  // O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s (log2 domain);
+  // the other pieces' partials were written by other CTAs of this launch: read them through L2
+  const int first = pm.x, S = pm.y;
+  const float* lse = p.ppart_lse + (size_t)first * kBM + row;
+  float M = -INFINITY;
+  for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(lse + (size_t)sp * kBM));
+  float den = 0.f;
+  for (int sp = 0; sp < S; ++sp) den += ex2(__ldcg(lse + (size_t)sp * kBM) - M);
+  const float dinv = 1.f / den;
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    float acc[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+#pragma unroll 1
+    for (int sp = 0; sp < S; ++sp) {
+      const float w = ex2(__ldcg(lse + (size_t)sp * kBM) - M);
+      const float4* src = reinterpret_cast<const float4*>(p.ppart_o + ((size_t)(first + sp) * kBM + row) * D + c * 32);
+      float4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = __ldcg(src + k);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        acc[4 * k] += w * v[k].x;
+        acc[4 * k + 1] += w * v[k].y;
+        acc[4 * k + 2] += w * v[k].z;
+        acc[4 * k + 3] += w * v[k].w;
       }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint4 v;
+      v.x = pack_bf16(acc[k * 8 + 0] * dinv, acc[k * 8 + 1] * dinv);
+      v.y = pack_bf16(acc[k * 8 + 2] * dinv, acc[k * 8 + 3] * dinv);
+      v.z = pack_bf16(acc[k * 8 + 4] * dinv, acc[k * 8 + 5] * dinv);
+      v.w = pack_bf16(acc[k * 8 + 6] * dinv, acc[k * 8 + 7] * dinv);
+      dst[k] = v;
     }
   }
   return true;
@@ -503,19 +623,27 @@ __device__ bool prefill_softmax(const PodParams& p, int4 it, uint8_t* smem, uint
 // O^T[d x 8] += V_page^T . P^T.  Pages arrive by TMA into a kNS-deep ring.
 // The block ids of an item's pages are read 32 at a time, one per lane, a
 // window ahead of use, so refilling a ring slot never waits on a global load.
-template <int D, int NS>
+template <int D, int NS, bool KV8>
 __device__ __forceinline__ void decode_issue_page(const PodParams& p, uint8_t* ring, uint64_t* wbars, uint32_t seq,
                                                   int blk, int kvh) {
   using CF = Cfg<D>;
+  constexpr int kStage = KV8 ? CF::kDecStage8 : CF::kDecStage;
+  constexpr int kPageB = KV8 ? CF::kPageBytes8 : CF::kPageBytes;
   const int s = seq % NS;
-  uint8_t* kbuf = ring + s * CF::kDecStage;
+  uint8_t* kbuf = ring + s * kStage;
   uint64_t* bar = &wbars[s];
-  mbar_arrive_expect_tx(bar, CF::kDecStage);
-  const int row = kv_row(p, blk, kvh);
-  // one box per page of K and of V: both 64-element halves of 16 rows land as
-  // [half][16 rows][128 B], the layout two 2D boxes would give
-  tma_load_3d(kbuf, &p.tm_kp, bar, 0, row, 0);
-  tma_load_3d(kbuf + CF::kPageBytes, &p.tm_vp, bar, 0, row, 0);
+  mbar_arrive_expect_tx(bar, kStage);
+  const int row = KV8 ? kv_row8(p, blk, kvh) : kv_row(p, blk, kvh);
+  if constexpr (KV8) {
+    // one box per e4m3 page of K and of V: 16 rows of d bytes (128-byte swizzle at d = 128)
+    tma_load_2d(kbuf, &p.tm_k8, bar, 0, row);
+    tma_load_2d(kbuf + kPageB, &p.tm_v8, bar, 0, row);
+  } else {
+    // one box per page of K and of V: both 64-element halves of 16 rows land as
+    // [half][16 rows][128 B], the layout two 2D boxes would give
+    tma_load_3d(kbuf, &p.tm_kp, bar, 0, row, 0);
+    tma_load_3d(kbuf + kPageB, &p.tm_vp, bar, 0, row, 0);
+  }
 }
 
 __device__ __forceinline__ uint32_t swz(int row, int col_elem) {
@@ -624,12 +752,44 @@ __device__ void merge_row_warp(const PodParams& p, int midx) {
   }
 }
 
-template <int D, int NS>
+// Score rows of the e4m3 decode page math.  Both m16n8k16 MMAs of a page
+// contract over a permuted order (a dot product does not depend on the order
+// of its terms, only on both operands using the same one):
+//  * d: in the S^T = K Q^T MMA, k-step ks = 4h + j (16 wide) gives lane q of a
+//    quad the four d values 64h + 16q + 4j .. +3, so one 16-byte shared load of
+//    a key row feeds four k-steps and the query fragment is read the same way;
+//  * keys: score row r of the 16-row tile is key sigma(r) of the page, chosen so
+//    that after the movmatrix transpose the P^T fragment of lane (n, q) holds
+//    keys sigma(2q), sigma(2q+1), sigma(2q+8), sigma(2q+9) = the 4q..4q+3 block,
+//    which is what one 32-bit load per key row of V provides;
+//  * in O^T = V^T P^T, the 16 output rows of M-tile 2p + t are d values
+//    32p + 4g + 2t (rows g) and 32p + 4g + 2t + 1 (rows g + 8).
+// sigma(r) = 4 q' + e + 2 (hi ^ (q' >> 1)) with q' = (r & 7) >> 1, e = r & 1,
+// hi = r >> 3: the 2-key blocks of lanes q >= 2 are swapped, which spreads the
+// four key rows one V load instruction touches over distinct swizzle phases.
+__device__ __forceinline__ int sigma_key(int r) {
+  const int qp = (r & 7) >> 1, e = r & 1, hi = r >> 3;
+  return 4 * qp + e + 2 * (hi ^ (qp >> 1));
+}
+
+// Byte offset of (row, byte b) of an e4m3 page in shared memory: rows of d
+// bytes, 16-byte chunks XOR-swizzled by the row at d = 128 (the tensor map's
+// 128-byte swizzle), plain at d = 64.
+template <int D>
+__device__ __forceinline__ uint32_t page8_off(int row, int b) {
+  if constexpr (D == 128) return (uint32_t)(row * 128 + ((((b >> 4) ^ row) & 7) << 4) + (b & 15));
+  else return (uint32_t)(row * D + b);
+}
+
+template <int D, int NS, bool KV8>
 __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, uint32_t& seq,
                             volatile int* abort_flag, int home_role) {
   using CF = Cfg<D>;
+  constexpr int kStage = KV8 ? CF::kDecStage8 : CF::kDecStage;
+  constexpr int kPageB = KV8 ? CF::kPageBytes8 : CF::kPageBytes;
   const int lane = threadIdx.x & 31;
   const int g = p.g;
+  const int gq = lane >> 2, q4 = lane & 3;   // quad row / lane within the quad
   while (true) {
     if (*abort_flag) return false;
     int item = 0;
@@ -652,7 +812,7 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
       const int pre = np < NS ? np : NS;
       for (int j = 0; j < pre; ++j) {
         const int blk = __shfl_sync(0xffffffffu, bt_cur, j);
-        if (lane == 0) decode_issue_page<D, NS>(p, ring, wbars, seq + j, blk, kvh);
+        if (lane == 0) decode_issue_page<D, NS, KV8>(p, ring, wbars, seq + j, blk, kvh);
       }
     }
     if (lane == 0) {
@@ -665,17 +825,33 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         atomicAdd(&e[3], 1);
       }
     }
-    // Q^T as the B operand: thread holds head n = lane/4, d pairs (lane%4)*2 (+8)
+    // Q^T as the B operand: lane holds head n = lane/4; bf16 pairs of d (lane%4)*2 (+8) per 16-wide
+    // step, or, for e4m3 pages, f16 pairs of d 64h + 16(lane%4) + 4j (+2) for step 4h + j
     uint32_t qf[D / 16][2];
+    const float sl2 = KV8 ? p.scale_log2 * __ldg(&p.k_scale8[kvh]) : p.scale_log2;
     {
-      const int n = lane >> 2;
-      const int dc = (lane & 3) * 2;
+      const int n = gq;
       if (n < g) {
         const __nv_bfloat16* qp = p.q_dec + ((size_t)r * p.Hq + kvh * g + n) * D;
+        if constexpr (KV8) {
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          qf[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + dc));
-          qf[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + dc));
+          for (int h = 0; h < D / 64; ++h) {
+            const uint4* src = reinterpret_cast<const uint4*>(qp + 64 * h + 16 * q4);
+            const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+            const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+              qf[4 * h + (i >> 1)][i & 1] = pack_f16(f.x, f.y);
+            }
+          }
+        } else {
+          const int dc = q4 * 2;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            qf[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + dc));
+            qf[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + dc));
+          }
         }
       } else {
 #pragma unroll
@@ -686,8 +862,10 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
     float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
-    const int key_lo = lane >> 2;     // S^T rows held: key_lo and key_lo + 8
-    // ldmatrix lane roles
+    // score rows held by this lane: keys key_lo and key_hi of the page
+    const int key_lo = KV8 ? sigma_key(gq) : gq;
+    const int key_hi = KV8 ? sigma_key(gq + 8) : gq + 8;
+    // ldmatrix lane roles (bf16 pages)
     const int a_row = lane & 15, a_colh = (lane >> 4) * 8;                  // K as A (non-trans)
     const int v_key = (lane & 7) + ((lane >> 4) << 3), v_colh = ((lane >> 3) & 1) * 8;  // V^T as A (trans)
     bool ok = true;
@@ -701,15 +879,20 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         jfail = j;
         break;
       }
-      uint8_t* kbuf = ring + s * CF::kDecStage;
-      uint8_t* vbuf = kbuf + CF::kPageBytes;
+      uint8_t* kbuf = ring + s * kStage;
+      uint8_t* vbuf = kbuf + kPageB;
       const int valid = min(kPage, k1 - (p0 + j) * kPage);
       if (valid < kPage) {
         // clear V rows past the end of the request: they may hold anything
-        for (int i = lane; i < (kPage - valid) * CF::kHalves * 8; i += 32) {
-          const int chunk = i & 7, rh = i >> 3;
-          const int key = valid + rh % (kPage - valid), h = rh / (kPage - valid);
-          *reinterpret_cast<uint4*>(vbuf + h * (kPage * 128) + key * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+        if constexpr (KV8) {
+          for (int i = lane; i < (kPage - valid) * (D / 16); i += 32)
+            *reinterpret_cast<uint4*>(vbuf + (valid + i / (D / 16)) * D + (i % (D / 16)) * 16) = make_uint4(0, 0, 0, 0);
+        } else {
+          for (int i = lane; i < (kPage - valid) * CF::kHalves * 8; i += 32) {
+            const int chunk = i & 7, rh = i >> 3;
+            const int key = valid + rh % (kPage - valid), h = rh / (kPage - valid);
+            *reinterpret_cast<uint4*>(vbuf + h * (kPage * 128) + key * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -718,20 +901,35 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
       // S^T = K Q^T over d in two independent accumulator chains (even and odd
       // 16-wide d slices), so the page's score latency is half a dependent chain
       float c[4] = {0.f, 0.f, 0.f, 0.f}, c2[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (KV8) {
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const int col = ks * 16 + a_colh;
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(kb_u + (col >> 6) * (kPage * 128) + swz(a_row, col & 63), a0, a1, a2, a3);
-        mma_16816((ks & 1) ? c2 : c, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+        for (int h = 0; h < D / 64; ++h) {
+          const uint4 ka = lds_u128(kb_u + page8_off<D>(key_lo, 64 * h + 16 * q4));
+          const uint4 kb = lds_u128(kb_u + page8_off<D>(key_hi, 64 * h + 16 * q4));
+          const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const int ks = 4 * h + jj;
+            mma_16816_f16((ks & 1) ? c2 : c, lo16_e4m3_to_f16x2(wa[jj]), lo16_e4m3_to_f16x2(wb[jj]),
+                          hi16_e4m3_to_f16x2(wa[jj]), hi16_e4m3_to_f16x2(wb[jj]), qf[ks][0], qf[ks][1]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int col = ks * 16 + a_colh;
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kb_u + (col >> 6) * (kPage * 128) + swz(a_row, col & 63), a0, a1, a2, a3);
+          mma_16816((ks & 1) ? c2 : c, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+        }
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) c[i] += c2[i];
       // mask, scale, online softmax per head (columns (lane%4)*2 and +1)
-      const float s0 = key_lo < valid ? c[0] * p.scale_log2 : -INFINITY;
-      const float s1 = key_lo < valid ? c[1] * p.scale_log2 : -INFINITY;
-      const float s2 = key_lo + 8 < valid ? c[2] * p.scale_log2 : -INFINITY;
-      const float s3 = key_lo + 8 < valid ? c[3] * p.scale_log2 : -INFINITY;
+      const float s0 = key_lo < valid ? c[0] * sl2 : -INFINITY;
+      const float s1 = key_lo < valid ? c[1] * sl2 : -INFINITY;
+      const float s2 = key_hi < valid ? c[2] * sl2 : -INFINITY;
+      const float s3 = key_hi < valid ? c[3] * sl2 : -INFINITY;
       float tA = fmaxf(s0, s2), tB = fmaxf(s1, s3);
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
@@ -745,18 +943,42 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
       const float e0 = ex2(s0 - nA), e1 = ex2(s1 - nB), e2 = ex2(s2 - nA), e3 = ex2(s3 - nB);
       lA = lA * alA + e0 + e2;
       lB = lB * alB + e1 + e3;
-      const uint32_t pb0 = movmatrix_t(pack_bf16(e0, e1));   // keys 0..7
-      const uint32_t pb1 = movmatrix_t(pack_bf16(e2, e3));   // keys 8..15
 #pragma unroll
       for (int mt = 0; mt < D / 16; ++mt) {
-        const int col = mt * 16 + v_colh;
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(vb_u + (col >> 6) * (kPage * 128) + swz(v_key, col & 63), a0, a1, a2, a3);
         acc[mt][0] *= alA;
         acc[mt][1] *= alB;
         acc[mt][2] *= alA;
         acc[mt][3] *= alB;
-        mma_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+      }
+      if constexpr (KV8) {
+        const uint32_t pb0 = movmatrix_t(pack_f16(e0, e1));   // score rows 0..7
+        const uint32_t pb1 = movmatrix_t(pack_f16(e2, e3));   // score rows 8..15
+        // this lane's V key rows sigma(2q), sigma(2q+1), sigma(2q+8), sigma(2q+9)
+        const int rot = 2 * (q4 >> 1);
+        const int ra = 4 * q4 + rot, rb = ra + 1, rc = 4 * q4 + (rot ^ 2), rd = rc + 1;
+#pragma unroll
+        for (int pg = 0; pg < D / 32; ++pg) {
+          const int col = 32 * pg + 4 * gq;
+          const uint32_t va = lds_u32(vb_u + page8_off<D>(ra, col)), vb = lds_u32(vb_u + page8_off<D>(rb, col));
+          const uint32_t vc = lds_u32(vb_u + page8_off<D>(rc, col)), vd = lds_u32(vb_u + page8_off<D>(rd, col));
+          // byte pairs (key a, key b) for d = col + 0/1 and col + 2/3
+          const uint32_t ab01 = __byte_perm(va, vb, 0x5140), ab23 = __byte_perm(va, vb, 0x7362);
+          const uint32_t cd01 = __byte_perm(vc, vd, 0x5140), cd23 = __byte_perm(vc, vd, 0x7362);
+          mma_16816_f16(acc[2 * pg], lo16_e4m3_to_f16x2(ab01), hi16_e4m3_to_f16x2(ab01), lo16_e4m3_to_f16x2(cd01),
+                        hi16_e4m3_to_f16x2(cd01), pb0, pb1);
+          mma_16816_f16(acc[2 * pg + 1], lo16_e4m3_to_f16x2(ab23), hi16_e4m3_to_f16x2(ab23),
+                        lo16_e4m3_to_f16x2(cd23), hi16_e4m3_to_f16x2(cd23), pb0, pb1);
+        }
+      } else {
+        const uint32_t pb0 = movmatrix_t(pack_bf16(e0, e1));   // keys 0..7
+        const uint32_t pb1 = movmatrix_t(pack_bf16(e2, e3));   // keys 8..15
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          const int col = mt * 16 + v_colh;
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vb_u + (col >> 6) * (kPage * 128) + swz(v_key, col & 63), a0, a1, a2, a3);
+          mma_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+        }
       }
       const int jn = j + NS;
       if (jn < np) {
@@ -768,7 +990,7 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         }
         const int blk = __shfl_sync(0xffffffffu, bt_cur, jn & 31);
         __syncwarp();
-        if (lane == 0) decode_issue_page<D, NS>(p, ring, wbars, sq + NS, blk, kvh);
+        if (lane == 0) decode_issue_page<D, NS, KV8>(p, ring, wbars, sq + NS, blk, kvh);
       }
     }
     if (!ok) {
@@ -791,38 +1013,69 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
       lA += __shfl_xor_sync(0xffffffffu, lA, o);
       lB += __shfl_xor_sync(0xffffffffu, lB, o);
     }
-    const int hA = (lane & 3) * 2, hB = hA + 1;
-    const float iA = 1.f / lA, iB = 1.f / lB;
-    const int d_lo = lane >> 2;
+    const int hA = q4 * 2, hB = hA + 1;
+    const float vsc = KV8 ? __ldg(&p.v_scale8[kvh]) : 1.f;
+    const float iA = vsc / lA, iB = vsc / lB;
     if (part < 0) {
       __nv_bfloat16* ob = p.o_dec + ((size_t)r * p.Hq + kvh * g) * D;
+      if constexpr (KV8) {
+        // M-tile 2pg + t holds d = 32 pg + 4 gq + 2t (+1 in rows gq + 8): four consecutive d per head
 #pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {
-        const int dd = mt * 16 + d_lo;
-        if (hA < g) {
-          ob[hA * D + dd] = __float2bfloat16_rn(acc[mt][0] * iA);
-          ob[hA * D + dd + 8] = __float2bfloat16_rn(acc[mt][2] * iA);
+        for (int pg = 0; pg < D / 32; ++pg) {
+          const int dd = 32 * pg + 4 * gq;
+          if (hA < g)
+            *reinterpret_cast<uint2*>(ob + hA * D + dd) =
+                make_uint2(pack_bf16(acc[2 * pg][0] * iA, acc[2 * pg][2] * iA),
+                           pack_bf16(acc[2 * pg + 1][0] * iA, acc[2 * pg + 1][2] * iA));
+          if (hB < g)
+            *reinterpret_cast<uint2*>(ob + hB * D + dd) =
+                make_uint2(pack_bf16(acc[2 * pg][1] * iB, acc[2 * pg][3] * iB),
+                           pack_bf16(acc[2 * pg + 1][1] * iB, acc[2 * pg + 1][3] * iB));
         }
-        if (hB < g) {
-          ob[hB * D + dd] = __float2bfloat16_rn(acc[mt][1] * iB);
-          ob[hB * D + dd + 8] = __float2bfloat16_rn(acc[mt][3] * iB);
+      } else {
+        const int d_lo = gq;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          const int dd = mt * 16 + d_lo;
+          if (hA < g) {
+            ob[hA * D + dd] = __float2bfloat16_rn(acc[mt][0] * iA);
+            ob[hA * D + dd + 8] = __float2bfloat16_rn(acc[mt][2] * iA);
+          }
+          if (hB < g) {
+            ob[hB * D + dd] = __float2bfloat16_rn(acc[mt][1] * iB);
+            ob[hB * D + dd + 8] = __float2bfloat16_rn(acc[mt][3] * iB);
+          }
         }
       }
     } else {
       float* po = p.part_o + (size_t)part * g * D;
+      if constexpr (KV8) {
 #pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {
-        const int dd = mt * 16 + d_lo;
-        if (hA < g) {
-          po[hA * D + dd] = acc[mt][0] * iA;
-          po[hA * D + dd + 8] = acc[mt][2] * iA;
+        for (int pg = 0; pg < D / 32; ++pg) {
+          const int dd = 32 * pg + 4 * gq;
+          if (hA < g)
+            *reinterpret_cast<float4*>(po + hA * D + dd) = make_float4(
+                acc[2 * pg][0] * iA, acc[2 * pg][2] * iA, acc[2 * pg + 1][0] * iA, acc[2 * pg + 1][2] * iA);
+          if (hB < g)
+            *reinterpret_cast<float4*>(po + hB * D + dd) = make_float4(
+                acc[2 * pg][1] * iB, acc[2 * pg][3] * iB, acc[2 * pg + 1][1] * iB, acc[2 * pg + 1][3] * iB);
         }
-        if (hB < g) {
-          po[hB * D + dd] = acc[mt][1] * iB;
-          po[hB * D + dd + 8] = acc[mt][3] * iB;
+      } else {
+        const int d_lo = gq;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          const int dd = mt * 16 + d_lo;
+          if (hA < g) {
+            po[hA * D + dd] = acc[mt][0] * iA;
+            po[hA * D + dd + 8] = acc[mt][2] * iA;
+          }
+          if (hB < g) {
+            po[hB * D + dd] = acc[mt][1] * iB;
+            po[hB * D + dd + 8] = acc[mt][3] * iB;
+          }
         }
       }
-      if (d_lo == 0) {
+      if (gq == 0) {
         if (hA < g) p.part_lse[(size_t)part * g + hA] = mA + __log2f(lA);
         if (hB < g) p.part_lse[(size_t)part * g + hB] = mB + __log2f(lB);
       }
@@ -846,12 +1099,13 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
 // Grid = SMs x CTAs/SM.  Each CTA takes one ticket from its SM's counter; the
 // ticket fixes its home role (prefill iff t mod (p+d) < p).  The CTA drains
 // its home queue, then the other one; no CTA ever waits for another.
-template <int D>
+template <int D, bool KV8>
 __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_constant__ PodParams p) {
   using CF = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + CF::kSmem);
-  uint32_t* ctrl = reinterpret_cast<uint32_t*>(bars + CF::kNumBars + 1);   // TMEM address, home role, item, abort
+  // TMEM address, home role, item, abort
+  uint32_t* ctrl = reinterpret_cast<uint32_t*>(bars + CF::kNumBars + 1);
   volatile int* sh_abort = reinterpret_cast<volatile int*>(ctrl + 3);
   const int tid = threadIdx.x, warp = tid >> 5;
   if (smem_u32(smem) & 1023u) {   // the swizzled tiles need 1024-byte alignment
@@ -869,6 +1123,10 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_kp);
     tma_prefetch_desc(&p.tm_vp);
+    if (KV8) {
+      tma_prefetch_desc(&p.tm_k8);
+      tma_prefetch_desc(&p.tm_v8);
+    }
     int home = p.mode == kDecodeOnly ? kRoleDecode : kRolePrefill;
     if (p.mode == kFused && p.partition_sms > 0) {
       // ablation: whole SMs start on one role (the first partition_sms SM ids prefill-first)
@@ -903,8 +1161,8 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
   // decode page rings: warp w < decode_warps owns ring w (ns stages) and its ns barriers
   const bool all_decode = p.decode_warps == kAllWarps;
   const int dwarps = all_decode ? kAllWarps : kWarpsPerCta;
-  const int ns = all_decode ? CF::kNSAll : CF::kNS;
-  uint8_t* ring = smem + (warp < dwarps ? warp : 0) * ns * CF::kDecStage;
+  const int ns = KV8 ? (all_decode ? CF::kNSAll8 : CF::kNS8) : (all_decode ? CF::kNSAll : CF::kNS);
+  uint8_t* ring = smem + (warp < dwarps ? warp : 0) * ns * (KV8 ? CF::kDecStage8 : CF::kDecStage);
   uint64_t* wbars = &bars[kBarDecode + (warp < dwarps ? warp : 0) * ns];
 
   for (int phase = 0; phase < 2; ++phase) {
@@ -924,11 +1182,11 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
           e[2] = home;
           atomicAdd(&e[3], 1);
         }
-        const int4 it = __ldg(&p.pre_items[item]);
+        const PreItem it = load_pre_item(p, item);
         bool ok;
         if (warp == kMmaWarp) ok = prefill_mma<D>(p, it, smem, bars, tmem, tiles_done, items_done);
         else if (warp == kTmaWarp) ok = prefill_tma<D>(p, it, smem, bars, tiles_done);
-        else ok = prefill_softmax<D>(p, it, smem, bars, tmem, tiles_done, items_done);
+        else ok = prefill_softmax<D>(p, it, item, smem, bars, tmem, tiles_done, items_done);
         tc_fence_before();
         const int fail = __syncthreads_or(!ok);
         tc_fence_after();
@@ -940,12 +1198,12 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
           __syncthreads();
           break;
         }
-        tiles_done += (uint32_t)((it.z + kBN - 1) / kBN);
+        tiles_done += (uint32_t)(it.j1 - it.j0);
         items_done += 1;
       }
     } else {
-      if (all_decode) decode_warp<D, CF::kNSAll>(p, ring, wbars, seq, sh_abort, home);
-      else if (warp < kWarpsPerCta) decode_warp<D, CF::kNS>(p, ring, wbars, seq, sh_abort, home);
+      if (all_decode) decode_warp<D, KV8 ? CF::kNSAll8 : CF::kNSAll, KV8>(p, ring, wbars, seq, sh_abort, home);
+      else if (warp < kWarpsPerCta) decode_warp<D, KV8 ? CF::kNS8 : CF::kNS, KV8>(p, ring, wbars, seq, sh_abort, home);
       __syncthreads();
     }
   }
@@ -1017,17 +1275,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int D>
+template <int D, bool KV8>
 int configure_kernels() {
-  static std::atomic<bool> done[64];   // per device; setting the attributes twice is harmless
+  static std::atomic<bool> done[64];   // per device and instantiation; setting the attributes twice is harmless
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 64 && done[dev].load(std::memory_order_acquire)) return POD_OK;
-  e = cudaFuncSetAttribute(pod_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemAlloc);
+  e = cudaFuncSetAttribute(pod_attn_kernel<D, KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Cfg<D>::kSmemAlloc);
   if (e != cudaSuccess) return cuda_fail(e);
   // two CTAs of ~113 KB need the whole 228 KB shared-memory carveout on every launch
-  e = cudaFuncSetAttribute(pod_attn_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+  e = cudaFuncSetAttribute(pod_attn_kernel<D, KV8>, cudaFuncAttributePreferredSharedMemoryCarveout,
                            (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 64) done[dev].store(true, std::memory_order_release);
@@ -1072,9 +1331,9 @@ int side_stream(SideStream** out) {
   return POD_OK;
 }
 
-template <int D>
+template <int D, bool KV8>
 int launch(const pod_attn_plan_t* pl, PodParams& prm, const MergeParams& mp, cudaStream_t st) {
-  int rc = configure_kernels<D>();
+  int rc = configure_kernels<D, KV8>();
   if (rc != POD_OK) return rc;
   const size_t smem = Cfg<D>::kSmemAlloc;
   if (pl->ev_start) cudaEventRecord(static_cast<cudaEvent_t>(pl->ev_start), st);
@@ -1083,12 +1342,12 @@ int launch(const pod_attn_plan_t* pl, PodParams& prm, const MergeParams& mp, cud
       prm.mode = kPrefillOnly;
       prm.use_tmem = 1;
       const int grid = pl->n_pre < pl->grid ? pl->n_pre : pl->grid;
-      pod_attn_kernel<D><<<grid, kThreads, smem, st>>>(prm);
+      pod_attn_kernel<D, KV8><<<grid, kThreads, smem, st>>>(prm);
     }
     if (pl->n_dec > 0) {
       prm.mode = kDecodeOnly;
       prm.use_tmem = 0;
-      pod_attn_kernel<D><<<pl->grid, kThreads, smem, st>>>(prm);
+      pod_attn_kernel<D, KV8><<<pl->grid, kThreads, smem, st>>>(prm);
     }
   } else if ((pl->cfg.flags & POD_FLAG_TWO_STREAMS) && pl->n_pre > 0 && pl->n_dec > 0) {
     SideStream* side = nullptr;
@@ -1101,17 +1360,17 @@ int launch(const pod_attn_plan_t* pl, PodParams& prm, const MergeParams& mp, cud
     prm.mode = kPrefillOnly;
     prm.use_tmem = 1;
     const int grid = pl->n_pre < pl->grid ? pl->n_pre : pl->grid;
-    pod_attn_kernel<D><<<grid, kThreads, smem, st>>>(prm);
+    pod_attn_kernel<D, KV8><<<grid, kThreads, smem, st>>>(prm);
     prm.mode = kDecodeOnly;
     prm.use_tmem = 0;
-    pod_attn_kernel<D><<<pl->grid, kThreads, smem, side->stream>>>(prm);
+    pod_attn_kernel<D, KV8><<<pl->grid, kThreads, smem, side->stream>>>(prm);
     e = cudaEventRecord(side->join, side->stream);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side->join, 0);
     if (e != cudaSuccess) return cuda_fail(e);
   } else if (pl->n_pre > 0 || pl->n_dec > 0) {
     prm.mode = kFused;
     prm.use_tmem = pl->n_pre > 0 ? 1 : 0;
-    pod_attn_kernel<D><<<pl->grid, kThreads, smem, st>>>(prm);
+    pod_attn_kernel<D, KV8><<<pl->grid, kThreads, smem, st>>>(prm);
   }
   if (pl->ev_stop) cudaEventRecord(static_cast<cudaEvent_t>(pl->ev_stop), st);
   if (pl->n_merge > 0 && (pl->cfg.flags & POD_FLAG_MERGE_KERNEL))
@@ -1191,12 +1450,21 @@ int pod_attn_plan_get_info(const pod_attn_plan_t* pl, pod_attn_plan_info* info) 
   info->table_bytes = (int64_t)pl->image.size();
   info->num_prefill_requests = pl->NP;
   info->num_prefill_rows = pl->P;
+  info->num_prefill_partials = pl->n_ppart;
+  info->num_prefill_merge_items = pl->n_pmerge;
+  info->rescale_count_offset = 4LL * kRescaleCount;
   return POD_OK;
 }
 
 int pod_attn_plan_prefill_requests(const pod_attn_plan_t* pl, int32_t* out) {
   if (!pl) return POD_ERR_INVALID_ARG;
   if (out && !pl->preq.empty()) std::memcpy(out, pl->preq.data(), pl->preq.size() * 4);
+  return POD_OK;
+}
+
+int pod_attn_plan_prefill_merges(const pod_attn_plan_t* pl, int32_t* out) {
+  if (!pl) return POD_ERR_INVALID_ARG;
+  if (out && !pl->pmerge.empty()) std::memcpy(out, pl->pmerge.data(), pl->pmerge.size() * 4);
   return POD_OK;
 }
 
@@ -1221,10 +1489,23 @@ int pod_attn_upload(const pod_attn_plan_t* pl, void* ws, size_t ws_bytes, void* 
   return POD_OK;
 }
 
-int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q_decode, const void* k_cache,
-                 const void* v_cache, int64_t num_blocks, const int32_t* block_table, int32_t block_table_stride,
-                 const int32_t* kv_lens, float scale, void* o_prefill, void* o_decode, void* ws, size_t ws_bytes,
-                 int32_t* trace, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The e4m3 cache of the decode requests (pod_attn_run_fp8kv).
+struct Fp8Args {
+  const void* k8;
+  const void* v8;
+  int64_t num_blocks8;
+  const float* k_scale;
+  const float* v_scale;
+};
+
+int run_impl(const pod_attn_plan_t* pl, const void* q_prefill, const void* q_decode, const void* k_cache,
+             const void* v_cache, int64_t num_blocks, const int32_t* block_table, int32_t block_table_stride,
+             const int32_t* kv_lens, float scale, void* o_prefill, void* o_decode, void* ws, size_t ws_bytes,
+             int32_t* trace, void* stream, const Fp8Args* f8) {
   if (!pl || !ws) return POD_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return POD_ERR_INVALID_ARG;
   if ((int64_t)ws_bytes < pl->ws_bytes) return POD_ERR_WORKSPACE;
@@ -1234,9 +1515,16 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
     return POD_ERR_INVALID_ARG;
   if (has_dec && (!q_decode || !o_decode || !aligned16(q_decode) || !aligned16(o_decode)))
     return POD_ERR_INVALID_ARG;
-  if ((has_pre || has_dec) &&
-      (!k_cache || !v_cache || !aligned16(k_cache) || !aligned16(v_cache) || !block_table || num_blocks < 1))
+  // the bf16 pools serve the prefill requests, and the decodes too unless an e4m3 cache is given
+  const bool need16 = has_pre || (has_dec && !f8);
+  if (need16 && (!k_cache || !v_cache || !aligned16(k_cache) || !aligned16(v_cache) || num_blocks < 1))
     return POD_ERR_INVALID_ARG;
+  if ((has_pre || has_dec) && !block_table) return POD_ERR_INVALID_ARG;
+  if (f8 && has_dec &&
+      (!f8->k8 || !f8->v8 || !aligned16(f8->k8) || !aligned16(f8->v8) || f8->num_blocks8 < 1 || !f8->k_scale ||
+       !f8->v_scale))
+    return POD_ERR_INVALID_ARG;
+  if (f8 && f8->num_blocks8 * Hkv * kPage >= (int64_t)INT32_MAX) return POD_ERR_UNSUPPORTED;
   if (block_table_stride < 1 || !(scale > 0.f) || scale != scale) return POD_ERR_INVALID_ARG;
   if (num_blocks * Hkv * kPage >= (int64_t)INT32_MAX) return POD_ERR_UNSUPPORTED;
   if ((pl->cfg.flags & POD_FLAG_TRACE) && !trace) return POD_ERR_INVALID_ARG;
@@ -1248,7 +1536,7 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
 
   PodParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  {
+  if (need16) {
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)num_blocks * Hkv * kPage};
     const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)kPage};
@@ -1270,6 +1558,23 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r3 != CUDA_SUCCESS || r4 != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
   }
+  if (f8 && has_dec) {
+    // e4m3 pages: rows of d bytes, one box {d, 16} per page (128-byte swizzle at d = 128)
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)f8->num_blocks8 * Hkv * kPage};
+    const cuuint64_t strides[1] = {(cuuint64_t)D};
+    const cuuint32_t box[2] = {(cuuint32_t)D, (cuuint32_t)kPage};
+    const cuuint32_t es[2] = {1, 1};
+    const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    CUresult r1 = enc(&prm.tm_k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(f8->k8), dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r2 = enc(&prm.tm_v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(f8->v8), dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r1 != CUDA_SUCCESS || r2 != CUDA_SUCCESS) return POD_ERR_INVALID_ARG;
+    prm.k_scale8 = f8->k_scale;
+    prm.v_scale8 = f8->v_scale;
+  }
   uint8_t* w = static_cast<uint8_t*>(ws);
   prm.q_pre = static_cast<const __nv_bfloat16*>(q_prefill);
   prm.q_dec = static_cast<const __nv_bfloat16*>(q_decode);
@@ -1283,6 +1588,10 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   prm.merge_items = reinterpret_cast<const int4*>(w + pl->off_merge);
   prm.pre_reqs = reinterpret_cast<const int4*>(w + pl->off_preq);
   prm.merge_cnt = reinterpret_cast<int32_t*>(w + pl->off_merge_cnt);
+  prm.pmerge_items = reinterpret_cast<const int4*>(w + pl->off_pmerge);
+  prm.pmerge_cnt = reinterpret_cast<int32_t*>(w + pl->off_pmerge_cnt);
+  prm.ppart_o = reinterpret_cast<float*>(w + pl->off_ppart_o);
+  prm.ppart_lse = reinterpret_cast<float*>(w + pl->off_ppart_lse);
   prm.merge_in_kernel = (pl->cfg.flags & POD_FLAG_MERGE_KERNEL) ? 0 : 1;
   prm.selftest_timeout = (pl->cfg.flags & POD_FLAG_SELFTEST_TIMEOUT) ? 1 : 0;
   prm.decode_warps = (pl->cfg.flags & POD_FLAG_DECODE_FOUR_WARPS) ? kWarpsPerCta : kAllWarps;
@@ -1297,6 +1606,10 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   prm.bt_stride = block_table_stride;
   prm.kv_rows = (int32_t)(num_blocks * Hkv * kPage);
   prm.num_blocks = (int32_t)num_blocks;
+  if (f8 && has_dec) {
+    prm.kv_rows8 = (int32_t)(f8->num_blocks8 * Hkv * kPage);
+    prm.num_blocks8 = (int32_t)f8->num_blocks8;
+  }
   prm.n_pre = pl->n_pre;
   prm.n_dec = pl->n_dec;
   prm.Hq = Hq;
@@ -1320,7 +1633,30 @@ int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q
   // counters (tickets, queue heads, error word, merge completions) start at zero every run
   cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)pl->off_pre, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  return D == 128 ? launch<128>(pl, prm, mp, st) : launch<64>(pl, prm, mp, st);
+  if (f8 && has_dec) return D == 128 ? launch<128, true>(pl, prm, mp, st) : launch<64, true>(pl, prm, mp, st);
+  return D == 128 ? launch<128, false>(pl, prm, mp, st) : launch<64, false>(pl, prm, mp, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pod_attn_run(const pod_attn_plan_t* pl, const void* q_prefill, const void* q_decode, const void* k_cache,
+                 const void* v_cache, int64_t num_blocks, const int32_t* block_table, int32_t block_table_stride,
+                 const int32_t* kv_lens, float scale, void* o_prefill, void* o_decode, void* ws, size_t ws_bytes,
+                 int32_t* trace, void* stream) {
+  return run_impl(pl, q_prefill, q_decode, k_cache, v_cache, num_blocks, block_table, block_table_stride, kv_lens,
+                  scale, o_prefill, o_decode, ws, ws_bytes, trace, stream, nullptr);
+}
+
+int pod_attn_run_fp8kv(const pod_attn_plan_t* pl, const void* q_prefill, const void* q_decode, const void* k_cache,
+                       const void* v_cache, int64_t num_blocks, const void* k_cache_fp8, const void* v_cache_fp8,
+                       int64_t num_blocks_fp8, const float* k_scale, const float* v_scale,
+                       const int32_t* block_table, int32_t block_table_stride, const int32_t* kv_lens, float scale,
+                       void* o_prefill, void* o_decode, void* ws, size_t ws_bytes, int32_t* trace, void* stream) {
+  const Fp8Args f8{k_cache_fp8, v_cache_fp8, num_blocks_fp8, k_scale, v_scale};
+  return run_impl(pl, q_prefill, q_decode, k_cache, v_cache, num_blocks, block_table, block_table_stride, kv_lens,
+                  scale, o_prefill, o_decode, ws, ws_bytes, trace, stream, &f8);
 }
 
 int pod_attn_plan_set_events(pod_attn_plan_t* pl, void* ev_start, void* ev_stop) {

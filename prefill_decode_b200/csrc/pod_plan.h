@@ -17,16 +17,22 @@ constexpr int kMaxSms = 512;         // ticket slots (smid is folded modulo this
 constexpr int kCostRatio = 248;      // B200 tensor FLOP/s per HBM byte/s (1624.7e12 / 6539.5e9)
 
 // Workspace layout (bytes).  Counters first, then one completion counter per
-// merge item (both zeroed every run); the tables follow in the order
-// prefill items | decode items | merge items | prefill requests; then split
-// partials.
+// decode merge item and per split prefill item (all zeroed every run); the
+// tables follow in the order prefill items | decode items | merge items |
+// prefill requests | prefill merge items; then the decode split partials
+// (O [n, g, d] and LSE [n, g], fp32) and the prefill piece partials
+// (O [n, 128, d] and LSE [n, 128], fp32).
 constexpr int64_t kCountersBytes = 4096;
 constexpr int kTicketBase = 0;       // int32 [kMaxSms]
 constexpr int kNextPrefill = 512;    // int32
 constexpr int kNextDecode = 513;     // int32
 constexpr int kErrorWord = 514;      // int32 (first error code recorded)
 constexpr int kErrorInfo = 515;      // int32 (item or block that caused it)
-constexpr int kPrefillItemInts = 4;  // q0 (within the request), q_head, kv_end, prefill request
+constexpr int kRescaleCount = 516;   // int32: prefill softmax warps that rescaled O (counted with POD_FLAG_TRACE)
+constexpr int kPrefillItemInts = 8;  // q0 (within the request), q_head, kv_end, prefill request,
+                                     // first and end key tile (64 keys each), partial (-1 = unsplit), merge
+constexpr int kPrefillMergeInts = 4; // first partial, pieces, 0, 0
+constexpr int kMaxPrefillPieces = 16; // KV pieces per prefill item at most
 constexpr int kPrefillReqInts = 4;   // q_start (row of q_prefill), P, C, 0
 constexpr int kMaxPrefillRequests = 4096;
 constexpr int kDecodeItemInts = 8;   // r, kv_head, k0, k1, partial, merge item, splits, 0
@@ -40,12 +46,15 @@ struct pod_attn_plan {
   pod_attn_config cfg;      // as given, with defaults resolved
   int32_t NP = 0, P = 0, B = 0, g = 1;   // prefill requests, their query rows in total, decodes
   int32_t n_pre = 0, n_dec = 0, n_merge = 0, n_part = 0;
+  int32_t n_ppart = 0, n_pmerge = 0;       // prefill partials and split prefill items
   int32_t ctas = 2, ratio_p = 1, ratio_d = 1, chunk_pages = 16, num_sms = 148, grid = 0;
-  int64_t off_merge_cnt = 0;   // int32 per merge item: splits finished (reset to 0 by the merging warp)
-  int64_t off_pre = 0, off_dec = 0, off_merge = 0, off_preq = 0, off_part_o = 0, off_part_lse = 0, ws_bytes = 0;
+  int64_t off_merge_cnt = 0;   // int32 per decode merge item: splits finished (zeroed every run)
+  int64_t off_pmerge_cnt = 0;  // int32 per split prefill item and softmax warp: pieces finished (zeroed every run)
+  int64_t off_pre = 0, off_dec = 0, off_merge = 0, off_preq = 0, off_pmerge = 0;
+  int64_t off_part_o = 0, off_part_lse = 0, off_ppart_o = 0, off_ppart_lse = 0, ws_bytes = 0;
   int64_t prefill_flops = 0, decode_flops = 0, kv_bytes = 0, qo_bytes = 0;
   std::vector<int32_t> decode_lens;
-  std::vector<int32_t> pre, dec, merge, preq;   // host tables
+  std::vector<int32_t> pre, dec, merge, preq, pmerge;   // host tables
   std::vector<uint8_t> image;                // host image of workspace [kCountersBytes, off_part_o)
   void* ev_start = nullptr;
   void* ev_stop = nullptr;

@@ -12,8 +12,6 @@
 // or any allocating routine.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "pod_plan.h"
 
 namespace {
@@ -21,26 +19,18 @@ namespace {
 // The workspace shared by every pod_attn_run_static call on a device.
 static __device__ __align__(256) unsigned char g_pod_static_scratch[POD_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
-
-// Device address of the scratch array for the current device, looked up once
-// per device.  In host code the array's name is only a host-side stand-in, so
-// the kernels must receive this address, never the name.
+// Device address of the scratch array in the current context.  In host code
+// the array's name is only a host-side stand-in, so the kernels must receive
+// this address, never the name.  It is looked up on every call rather than
+// cached: after cudaDeviceReset (or in another context on the same device) the
+// module is loaded again and the array may sit elsewhere, and a cached address
+// would then point at unmapped memory.  Once the module is loaded in the
+// context the lookup is a table read, not a stream operation.
 int scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return POD_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return POD_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_pod_static_scratch);
-    if (e != cudaSuccess || !p) return POD_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_pod_static_scratch);
+  if (e != cudaSuccess || !p) return POD_ERR_CUDA;
+  *out = p;
   return POD_OK;
 }
 

@@ -1,5 +1,9 @@
-"""Test/bench helper: move a synthetic batch to the GPU and run it through the
-C ABI.  Marshalling only (torch allocates device memory); no attention math."""
+"""Device copies of a synthetic hybrid batch, run through the C ABI.
+
+Marshalling only: torch allocates the device tensors (Q, the paged K/V pools,
+block table, lengths, outputs, workspace) and the calls go through the
+binding's Plan; there is no attention arithmetic here.  Used by the tests,
+``bench.py`` and ``__graft_entry__.smoke()``."""
 from __future__ import annotations
 
 import numpy as np
@@ -99,6 +103,45 @@ class DeviceBatch:
         op = self.o_pre.float().cpu().numpy().astype(np.float64) if self.o_pre is not None else None
         od = self.o_dec.float().cpu().numpy().astype(np.float64) if self.o_dec is not None else None
         return op, od
+
+    # ------------------------------------------------------------ e4m3 cache
+    def attach_fp8(self, cache, device=None):
+        """Device copies of an e4m3 cache made on the host (synth.fp8_cache)."""
+        dev = self.k.device if device is None else device
+        t = self.torch
+        self.k8 = t.from_numpy(cache.k_pool).to(dev)
+        self.v8 = t.from_numpy(cache.v_pool).to(dev)
+        self.k_scale = t.from_numpy(cache.k_scale).to(dev)
+        self.v_scale = t.from_numpy(cache.v_scale).to(dev)
+        return self
+
+    def fp8_on_device(self):
+        """An e4m3 copy of the device pools made on the GPU (large batches): per kv head,
+        scale = largest |value| outside the poison / 448; codes = the value / scale, clamped to
+        +-448 and converted by torch (round to nearest even); poison slots get +448 (K) and
+        -448 (V).  Input preparation only; the kernel sees nothing but the codes and scales."""
+        import synth
+        t = self.torch
+        out = []
+        for pool, poison, code in ((self.k, synth.POISON_K, synth.POISON_E4M3_K),
+                                   (self.v, synth.POISON_V, synth.POISON_E4M3_V)):
+            f = pool.float()
+            bad = f == poison
+            amax = t.where(bad, t.zeros_like(f), f.abs()).amax(dim=(0, 2, 3))
+            scale = (amax / synth.E4M3_MAX).clamp_min(1e-8).to(t.float32)
+            q = (f / scale[None, :, None, None]).clamp(-synth.E4M3_MAX, synth.E4M3_MAX)
+            q = q.to(t.float8_e4m3fn).view(t.uint8)
+            q[bad] = code
+            out.append((q.contiguous(), scale))
+            del f, bad
+        (self.k8, self.k_scale), (self.v8, self.v_scale) = out
+        return self
+
+    def run_fp8(self, pod, plan, ws, trace=None, stream=None):
+        """pod_attn_run_fp8kv: decodes read the e4m3 copy (same block table), prefill the bf16 pools."""
+        plan.run_fp8kv(self.q_pre, self.q_dec, self.k, self.v, self.b.num_blocks, self.k8, self.v8,
+                       self.k8.shape[0], self.k_scale, self.v_scale, self.bt, self.bt.shape[1], self.lens,
+                       self.b.scale, self.o_pre, self.o_dec, ws, trace=trace, stream=stream)
 
     def error_word(self, plan, ws):
         off = plan.info.error_offset

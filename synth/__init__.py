@@ -61,6 +61,31 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
     return bf16_bits_to_f32(b).astype(np.float64)
 
 
+E4M3_MAX = 448.0
+
+
+def f64_to_e4m3_bits(v: np.ndarray) -> np.ndarray:
+    """float64 -> e4m3 byte (uint8): round to nearest, ties to even, saturating at +-448.
+
+    Input generation only (the FP8 cache is made from the bf16 values); the
+    decoding that both sides compute with is the format's own definition."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    # quantum of the binade: 2^(e-3) for normals (|v| >= 2^-6), 2^-9 below
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))           # a = f 2^ex, f in [0.5, 1)
+    e = np.clip(ex - 1, -6, 8)
+    quantum = np.ldexp(1.0, (e - 3).astype(np.int64))
+    q = np.minimum(np.rint(a / quantum) * quantum, E4M3_MAX)
+    _, qx = np.frexp(np.where(q > 0, q, 1.0))
+    qe = qx - 1
+    normal = q >= 2.0 ** -6
+    ebits = np.where(normal, qe + 7, 0)
+    mant = np.where(normal, q / np.ldexp(1.0, qe.astype(np.int64)) * 8 - 8, q / 2.0 ** -9)
+    bits = (ebits.astype(np.int64) << 3) | np.rint(mant).astype(np.int64)
+    bits = np.where(np.signbit(v), bits | 0x80, bits)
+    return bits.astype(np.uint8)
+
+
 def _normal_bf16(rng: np.random.Generator, shape: Sequence[int]) -> np.ndarray:
     n = int(np.prod(shape, dtype=np.int64))
     out = np.empty(n, dtype=np.uint16)
@@ -226,6 +251,40 @@ def make_batch(w: Workload) -> Batch:
         k_pool[blk] = pk
         v_pool[blk] = pv
     return Batch(w, q_pre, q_dec, k_pool, v_pool, bt, kv_lens, w.softmax_scale)
+
+
+@dataclasses.dataclass
+class Fp8Cache:
+    """The same paged cache stored as e4m3 bytes with one fp32 scale per kv head for K
+    and for V; read by the decode requests (block-table rows from NP on)."""
+    k_pool: np.ndarray        # uint8 [num_blocks, Hkv, 16, d]
+    v_pool: np.ndarray        # uint8 [num_blocks, Hkv, 16, d]
+    k_scale: np.ndarray       # float32 [Hkv]
+    v_scale: np.ndarray       # float32 [Hkv]
+
+
+POISON_E4M3_K = 0x7E          # +448: unused slots and blocks, as in the bf16 pools
+POISON_E4M3_V = 0xFE          # -448
+
+
+def fp8_cache(b: Batch) -> Fp8Cache:
+    """Quantise a batch's K/V pools to e4m3 (no random draws: derived from the bf16 values).
+
+    Scale of kv head h = (largest |value| of that head's pool outside the poison) / 448,
+    rounded to float32; bytes = RNE(value / scale) saturated at 448; poison slots and
+    blocks hold +448 (K) and -448 (V)."""
+    out = []
+    for pool, poison_bf16, poison8 in ((b.k_pool, POISON_K, POISON_E4M3_K), (b.v_pool, POISON_V, POISON_E4M3_V)):
+        f = bf16_bits_to_f32(pool).astype(np.float64)
+        is_poison = f == poison_bf16
+        amax = np.where(is_poison, 0.0, np.abs(f)).max(axis=(0, 2, 3))
+        scale = np.maximum(amax / E4M3_MAX, 1e-8).astype(np.float32)
+        q = np.empty(pool.shape, dtype=np.uint8)
+        for h in range(pool.shape[1]):
+            q[:, h] = f64_to_e4m3_bits(f[:, h] / np.float64(scale[h]))
+        q[is_poison] = poison8
+        out.append((q, scale))
+    return Fp8Cache(out[0][0], out[1][0], out[0][1], out[1][1])
 
 
 # ---------------------------------------------------------------------------

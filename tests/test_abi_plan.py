@@ -51,19 +51,35 @@ def _lens(w):
     return [int(x) for x in synth._draw_lengths(np.random.default_rng(w.seed), w)]
 
 
-def _compare(pod, Hq, Hkv, d, sms, P, KV, lens, **kw):
-    ref = plan_ref(Hq, Hkv, d, sms, P, KV, lens, **kw)
+def _c_plan(pod, Hq, Hkv, d, sms, P, KV, lens, **kw):
+    """The same batch and knobs through the C planner (keyword names as plan_ref's)."""
     ratio = (kw.get("ratio_p", 0), kw.get("ratio_d", 0))
     flags = pod.POD_FLAG_DECODE_FOUR_WARPS if kw.get("decode_warps", 6) == 4 else 0
-    pl = pod.Plan(Hq, Hkv, d, P, KV, lens, num_sms=sms, ctas_per_sm=kw.get("ctas_per_sm", 0), ratio=ratio,
-                  max_waves=kw.get("max_waves", 0), min_chunk_pages=kw.get("min_chunk_pages", 0), flags=flags)
+    if kw.get("split_unlimited", False):
+        flags |= pod.POD_FLAG_PREFILL_SPLIT_UNLIMITED
+    return pod.Plan(Hq, Hkv, d, P, KV, lens, num_sms=sms, ctas_per_sm=kw.get("ctas_per_sm", 0), ratio=ratio,
+                    max_waves=kw.get("max_waves", 0), min_chunk_pages=kw.get("min_chunk_pages", 0),
+                    max_prefill_splits=kw.get("prefill_splits", 0), flags=flags)
+
+
+def _same_tables(pl, ref):
     pre, dec, mer = pl.tables()
     np.testing.assert_array_equal(pre, ref.prefill_items)
     np.testing.assert_array_equal(dec, ref.decode_items)
     np.testing.assert_array_equal(mer, ref.merge_items)
+    np.testing.assert_array_equal(pl.prefill_merges(), ref.prefill_merge_items)
     i = pl.info
     assert (i.ctas_per_sm, i.ratio_prefill, i.ratio_decode, i.chunk_pages, i.num_partials) == (
         ref.ctas_per_sm, ref.ratio_p, ref.ratio_d, ref.chunk_pages, ref.num_partials)
+    assert (i.num_prefill_items, i.num_prefill_partials, i.num_prefill_merge_items) == (
+        len(ref.prefill_items), ref.num_prefill_partials, len(ref.prefill_merge_items))
+
+
+def _compare(pod, Hq, Hkv, d, sms, P, KV, lens, **kw):
+    ref = plan_ref(Hq, Hkv, d, sms, P, KV, lens, **kw)
+    pl = _c_plan(pod, Hq, Hkv, d, sms, P, KV, lens, **kw)
+    _same_tables(pl, ref)
+    i = pl.info
     assert i.grid == sms * ref.ctas_per_sm
     return pl
 
@@ -91,7 +107,8 @@ def test_c_plan_matches_plan_ref_random(pod):
         kw = dict(ctas_per_sm=int(rng.choice([0, 1, 2])), max_waves=int(rng.choice([0, 1, 3])),
                   min_chunk_pages=int(rng.choice([0, 1, 4, 16])),
                   ratio_p=int(rng.choice([0, 0, 1, 2])), ratio_d=int(rng.choice([0, 0, 1, 3])),
-                  decode_warps=int(rng.choice([4, 6])))
+                  decode_warps=int(rng.choice([4, 6])), prefill_splits=int(rng.choice([0, 0, 1, 2, 5, 16])),
+                  split_unlimited=bool(rng.integers(0, 2)))
         _compare(pod, Hkv * g, Hkv, int(rng.choice([64, 128])), int(rng.integers(1, 200)), P, C + P, lens, **kw)
 
 
@@ -114,18 +131,10 @@ def test_c_plan_rejects(pod, bad, code):
 
 def _compare_batched(pod, Hq, Hkv, d, sms, qo, kv, lens, **kw):
     ref = plan_ref_batched(Hq, Hkv, d, sms, qo, kv, lens, **kw)
-    ratio = (kw.get("ratio_p", 0), kw.get("ratio_d", 0))
-    flags = pod.POD_FLAG_DECODE_FOUR_WARPS if kw.get("decode_warps", 6) == 4 else 0
-    pl = pod.Plan(Hq, Hkv, d, qo, kv, lens, num_sms=sms, ctas_per_sm=kw.get("ctas_per_sm", 0), ratio=ratio,
-                  max_waves=kw.get("max_waves", 0), min_chunk_pages=kw.get("min_chunk_pages", 0), flags=flags)
-    pre, dec, mer = pl.tables()
-    np.testing.assert_array_equal(pre, ref.prefill_items)
-    np.testing.assert_array_equal(dec, ref.decode_items)
-    np.testing.assert_array_equal(mer, ref.merge_items)
+    pl = _c_plan(pod, Hq, Hkv, d, sms, qo, kv, lens, **kw)
+    _same_tables(pl, ref)
     np.testing.assert_array_equal(pl.prefill_requests(), ref.prefill_requests)
     i = pl.info
-    assert (i.ctas_per_sm, i.ratio_prefill, i.ratio_decode, i.chunk_pages, i.num_partials) == (
-        ref.ctas_per_sm, ref.ratio_p, ref.ratio_d, ref.chunk_pages, ref.num_partials)
     assert (i.num_prefill_requests, i.num_prefill_rows) == (len(qo), sum(qo))
     # algorithmic counts over every prefill request
     assert i.prefill_flops == 4 * d * Hq * sum(sum(K - P + j + 1 for j in range(P)) for P, K in zip(qo, kv))
@@ -144,7 +153,8 @@ def test_c_batched_plan_matches_plan_ref_random(pod):
         kv = [P + (int(rng.integers(0, 3000)) if P else int(rng.integers(0, 5))) for P in qo]
         lens = [int(x) for x in rng.integers(1, 6000, size=int(rng.integers(0, 30)))]
         kw = dict(ctas_per_sm=int(rng.choice([0, 1, 2])), max_waves=int(rng.choice([0, 1, 3])),
-                  min_chunk_pages=int(rng.choice([0, 1, 16])), decode_warps=int(rng.choice([4, 6])))
+                  min_chunk_pages=int(rng.choice([0, 1, 16])), decode_warps=int(rng.choice([4, 6])),
+                  prefill_splits=int(rng.choice([0, 0, 1, 3])), split_unlimited=bool(rng.integers(0, 2)))
         _compare_batched(pod, Hkv * g, Hkv, int(rng.choice([64, 128])), int(rng.integers(1, 200)), qo, kv, lens, **kw)
 
 
@@ -232,7 +242,8 @@ def test_c_planner_matches_plan_ref_property(pod):
         sms=st.integers(1, 300), chunks=st.lists(chunk, max_size=5),
         lens=st.lists(st.integers(1, 40000), max_size=40),
         ctas=st.sampled_from([0, 1, 2]), waves=st.integers(0, 4), minc=st.integers(0, 40),
-        rp=st.integers(0, 3), rd=st.integers(0, 3), dw=st.sampled_from([4, 6])))
+        rp=st.integers(0, 3), rd=st.integers(0, 3), dw=st.sampled_from([4, 6]),
+        ps=st.sampled_from([0, 1, 2, 4, 16, 17]), unl=st.booleans()))
 
     @settings(max_examples=150, deadline=None, suppress_health_check=[HealthCheck.too_slow])
     @given(batch)
@@ -240,16 +251,15 @@ def test_c_planner_matches_plan_ref_property(pod):
         qo = [P for P, _ in x["chunks"]]
         kv = [P + C if P else C % 3 for P, C in x["chunks"]]
         kw = dict(ctas_per_sm=x["ctas"], max_waves=x["waves"], min_chunk_pages=x["minc"],
-                  ratio_p=x["rp"], ratio_d=x["rd"], decode_warps=x["dw"])
+                  ratio_p=x["rp"], ratio_d=x["rd"], decode_warps=x["dw"], prefill_splits=x["ps"],
+                  split_unlimited=x["unl"])
         try:
             ref = plan_ref_batched(x["Hkv"] * x["g"], x["Hkv"], x["d"], x["sms"], qo, kv, x["lens"], **kw)
         except PlanError:
             ref = None
         if ref is None:
             with pytest.raises(pod.PodError):
-                pod.Plan(x["Hkv"] * x["g"], x["Hkv"], x["d"], qo, kv, x["lens"], num_sms=x["sms"],
-                         ctas_per_sm=x["ctas"], ratio=(x["rp"], x["rd"]), max_waves=x["waves"],
-                         min_chunk_pages=x["minc"], flags=pod.POD_FLAG_DECODE_FOUR_WARPS if x["dw"] == 4 else 0)
+                _c_plan(pod, x["Hkv"] * x["g"], x["Hkv"], x["d"], x["sms"], qo, kv, x["lens"], **kw)
             return
         _compare_batched(pod, x["Hkv"] * x["g"], x["Hkv"], x["d"], x["sms"], qo, kv, x["lens"], **kw)
 

@@ -10,7 +10,7 @@ import pytest
 
 import synth
 from oracle import attention as A
-from tests.podrun import DeviceBatch
+from prefill_decode_b200.device_batch import DeviceBatch
 
 pytestmark = pytest.mark.gpu
 
@@ -208,3 +208,58 @@ def test_repeat_runs_are_stable(env):
         db.run(pod, pl, ws)
     torch.cuda.synchronize()
     assert torch.equal(first[0], db.o_pre) and torch.equal(first[1], db.o_dec)
+
+
+# ----------------------------------------------------------- prefill KV pieces
+# Batches whose prefill items the plan cuts into KV pieces (merged by the CTA that finishes the
+# item's last piece): d = 64 / 128, g = 1..8, ragged chunk ends, no prior context, several requests.
+SPLIT = [
+    synth.custom("split_d128_g4", 8, 2, 128, 300, 2500, [17, 1000, 3000], 40),
+    synth.custom("split_d64_g2_prefill_only", 4, 2, 64, 70, 1800, [], 41),
+    synth.custom("split_mha_g1", 4, 4, 128, 129, 1600, [33], 42),
+    synth.custom("split_g8", 16, 2, 128, 64, 3000, [5000, 17], 43),
+    synth.custom("split_g3_d64", 6, 2, 64, 200, 1200, [700], 44),
+    synth.custom("split_g5", 10, 2, 128, 100, 900, [2600, 17], 45),
+    synth.custom("split_g7", 28, 4, 128, 96, 1500, [3500, 1], 46),
+    synth.custom("split_no_prior", 8, 2, 128, 1200, 0, [100, 900], 47),
+    synth.custom_batched("split_batched", 8, 2, 128, [(300, 2000), (1, 900), (0, 0), (129, 3000)], [1, 1000], 48),
+]
+
+
+@pytest.mark.parametrize("w", SPLIT, ids=lambda w: w.name)
+@pytest.mark.parametrize("flags", [0, 1, 16, 64], ids=["fused", "sequential", "two_streams", "four_warps"])
+def test_split_prefill_full_parity(env, w, flags):
+    b = synth.make_batch(w)
+    db, pl, ws = _run(env, b, flags=flags)
+    assert pl.info.num_prefill_partials > 0, "the batch should split its prefill"
+    op, od = db.outputs()
+    rp, rd = _oracle(b)
+    _check(op, rp, f"{w.name} prefill")
+    if rd is not None:
+        _check(od, rd, f"{w.name} decode")
+
+
+@pytest.mark.parametrize("kw", [dict(max_prefill_splits=2), dict(max_prefill_splits=16), dict(max_prefill_splits=1),
+                                dict(flags=128), dict(flags=128 | 1), dict(flags=128, ctas_per_sm=1),
+                                dict(flags=128, ratio=(0, 1)), dict(flags=128 | 32)],
+                         ids=["cap2", "cap16", "never", "unlimited", "unlimited_sequential", "unlimited_one_cta",
+                              "unlimited_decode_first", "unlimited_sm_partition"])
+def test_split_knobs_keep_results(env, kw):
+    w = synth.custom("split_knobs", 8, 2, 128, 300, 1700, [16, 1000, 2500, 4096], 49)
+    b = synth.make_batch(w)
+    db, pl, ws = _run(env, b, **kw)
+    if kw.get("max_prefill_splits") != 1:
+        assert pl.info.num_prefill_partials > 0
+    op, od = db.outputs()
+    rp, rd = _oracle(b)
+    _check(op, rp, "prefill")
+    _check(od, rd, "decode")
+
+
+def test_llama3_8b_mix_sampled_unlimited_split(env):
+    """The full-size bench batch with the co-located limit off: 256 prefill pieces merged in-kernel."""
+    torch, pod = env
+    w = synth.llama3_8b_mix()
+    db, pl, ws, b = _sampled(env, w, [0, 1, 127, 128, 255, 256, 383, 384, 510, 511], [0, 31, 63],
+                             flags=pod.POD_FLAG_PREFILL_SPLIT_UNLIMITED)
+    assert pl.info.num_prefill_partials == 256

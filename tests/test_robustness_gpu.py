@@ -12,7 +12,7 @@ import pytest
 
 import synth
 from oracle import attention as A
-from tests.podrun import DeviceBatch
+from prefill_decode_b200.device_batch import DeviceBatch
 
 pytestmark = pytest.mark.gpu
 

@@ -9,7 +9,8 @@ import numpy as np
 import pytest
 
 import synth
-from tests.podrun import DeviceBatch
+from oracle import attention as A
+from prefill_decode_b200.device_batch import DeviceBatch
 
 pytestmark = pytest.mark.gpu
 
@@ -32,20 +33,30 @@ def _close(a, b):
     return np.isfinite(a).all() and e.max() <= MAX_ABS and e.mean() <= MEAN_ABS
 
 
-def test_static_scratch_matches_workspace_entry_point(env):
+@pytest.mark.parametrize("heads", [(32, 8), (8, 2)], ids=["decode_splits", "decode_and_prefill_splits"])
+def test_static_scratch_matches_workspace_entry_point(env, heads):
     torch, pod = env
-    # splits (partials + merge) and a ragged multi-tile prefill, so the scratch is really used
-    w = synth.custom("no_alloc", 32, 8, 128, 300, 900, [17, 1000, 3000, 5000, 257], 21)
+    # decode splits (partials + merge) and a ragged multi-tile prefill, so the scratch is really used;
+    # with 8/2 heads the prefill items are cut into KV pieces too, whose partials also live there
+    Hq, Hkv = heads
+    w = synth.custom("no_alloc", Hq, Hkv, 128, 300, 900, [17, 1000, 3000, 5000, 257], 21)
     b = synth.make_batch(w)
     db = DeviceBatch(torch, b)
     plan = db.plan(pod, max_waves=8)
     assert plan.info.num_partials > 0
+    assert (plan.info.num_prefill_partials > 0) == (Hq == 8)
     assert plan.workspace_bytes <= (8 << 20)
     ws = db.workspace(plan)
     plan.upload(ws)
     db.run(pod, plan, ws)
     torch.cuda.synchronize()
     ref_pre, ref_dec = db.outputs()
+
+    w = b.workload
+    ora_pre = A.attend_prefill(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_ctx, b.scale,
+                               w.num_kv_heads)
+    ora_dec = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, w.num_kv_heads)
+    assert _close(ref_pre, ora_pre) and _close(ref_dec, ora_dec)
 
     L = pod.lib()
     for call in range(2):
@@ -60,6 +71,9 @@ def test_static_scratch_matches_workspace_entry_point(env):
         got_pre, got_dec = db.outputs()
         assert _close(got_pre, ref_pre), f"call {call}: prefill differs"
         assert _close(got_dec, ref_dec), f"call {call}: decode differs"
+        # and against the float64 oracle, at the tolerance of every other parity test
+        assert _close(got_pre, ora_pre), f"call {call}: prefill differs from the oracle"
+        assert _close(got_dec, ora_dec), f"call {call}: decode differs from the oracle"
 
 
 def test_static_scratch_rejects_oversized_plan(env):
