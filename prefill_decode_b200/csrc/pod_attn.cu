@@ -1120,9 +1120,11 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
     }
     fence_mbar_init();
     *sh_abort = 0;
-    tma_prefetch_desc(&p.tm_k);
-    tma_prefetch_desc(&p.tm_kp);
-    tma_prefetch_desc(&p.tm_vp);
+    if (!KV8 || p.n_pre > 0) {   // with an e4m3 cache and no prefill the bf16 maps are not encoded
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_kp);
+      tma_prefetch_desc(&p.tm_vp);
+    }
     if (KV8) {
       tma_prefetch_desc(&p.tm_k8);
       tma_prefetch_desc(&p.tm_v8);

@@ -168,3 +168,38 @@ def test_out_of_range_block_id_in_a_batched_prefill_request(env):
     rd = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, 2, first_row=2)
     assert _close(od, rd)
     assert np.isfinite(op[100:]).all()
+
+
+def test_split_prefill_trace_and_bad_block(env):
+    """With prefill items cut into KV pieces every piece runs exactly once (trace), and a bad
+    block id inside one piece is reported in the error word; the decodes stay correct."""
+    torch, pod = env
+    w = synth.custom("robust_split", 8, 2, 128, 256, 2000, [300, 1200], 34)
+    b = synth.make_batch(w)
+    db = DeviceBatch(torch, b)
+    pl = db.plan(pod, flags=pod.POD_FLAG_TRACE)
+    assert pl.info.num_prefill_partials > 0
+    ws = db.workspace(pl)
+    pl.upload(ws)
+    n = pl.info.num_prefill_items + pl.info.num_decode_items
+    trace = torch.zeros(n * 4, dtype=torch.int32, device="cuda")
+    db.run(pod, pl, ws, trace=trace)
+    torch.cuda.synchronize()
+    assert db.error_word(pl, ws) == 0
+    assert (trace.view(n, 4)[:, 3] == 1).all().item()
+    rp = A.attend_prefill(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_ctx, b.scale, 2)
+    assert _close(db.outputs()[0], rp)
+    # now a bad block id on page 40 (keys 640..655) of the prefill request
+    bt = b.block_table.copy()
+    bt[0, 40] = 10 ** 6
+    db.bt = torch.from_numpy(bt).cuda()
+    pl2 = db.plan(pod)
+    ws2 = db.workspace(pl2)
+    pl2.upload(ws2)
+    db.run(pod, pl2, ws2)
+    torch.cuda.synchronize()
+    assert db.error_word(pl2, ws2) == pod.POD_ERR_BOUNDS
+    op, od = db.outputs()
+    assert np.isfinite(op).all()
+    rd = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, 2)
+    assert _close(od, rd)
