@@ -230,16 +230,13 @@ template <int D>
 __device__ __forceinline__ void issue_tile(const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int row_lane,
                                            int lane) {
   using CF = Cfg<D>;
-  int rows[kBN / kPage];
+  // lanes 0-3 each issue the boxes of one page (row_lane of lane l is page l & 3)
+  if (lane == 0) mbar_arrive_expect_tx(bar, CF::kKTile);
+  __syncwarp();
+  if (lane < kBN / kPage) {
 #pragma unroll
-  for (int pi = 0; pi < kBN / kPage; ++pi) rows[pi] = __shfl_sync(0xffffffffu, row_lane, pi);
-  if (lane == 0) {
-    mbar_arrive_expect_tx(bar, CF::kKTile);
-#pragma unroll
-    for (int pi = 0; pi < kBN / kPage; ++pi)
-#pragma unroll
-      for (int h = 0; h < CF::kHalves; ++h)
-        tma_load_2d(dst + h * (kBN * 128) + pi * (kPage * 128), map, bar, h * 64, rows[pi]);
+    for (int h = 0; h < CF::kHalves; ++h)
+      tma_load_2d(dst + h * (kBN * 128) + lane * (kPage * 128), map, bar, h * 64, row_lane);
   }
 }
 
@@ -249,14 +246,9 @@ __device__ __forceinline__ void issue_tile(const CUtensorMap* map, uint8_t* dst,
 template <int D>
 __device__ __forceinline__ void issue_vtile(const PodParams& p, uint8_t* dst, uint64_t* bar, int row_lane, int lane) {
   using CF = Cfg<D>;
-  int rows[kBN / kPage];
-#pragma unroll
-  for (int pi = 0; pi < kBN / kPage; ++pi) rows[pi] = __shfl_sync(0xffffffffu, row_lane, pi);
-  if (lane == 0) {
-    mbar_arrive_expect_tx(bar, CF::kKTile);
-#pragma unroll
-    for (int pi = 0; pi < kBN / kPage; ++pi) tma_load_3d(dst + pi * CF::kPageBytes, &p.tm_vp, bar, 0, rows[pi], 0);
-  }
+  if (lane == 0) mbar_arrive_expect_tx(bar, CF::kKTile);
+  __syncwarp();
+  if (lane < kBN / kPage) tma_load_3d(dst + lane * CF::kPageBytes, &p.tm_vp, bar, 0, row_lane, 0);
 }
 
 // TMA warp of one prefill item: K into a 3-deep ring and V into a 2-deep
