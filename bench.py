@@ -513,10 +513,19 @@ def main():
         # parity spot check of the e4m3 run against the float64 oracle on the same codes
         from oracle import attention as A8, fp8 as F8
         reqs8 = [0, w.num_decode // 2, w.num_decode - 1]
-        K8 = F8.dequant_pool(db.k8.cpu().numpy(), db.k_scale.cpu().numpy())
-        V8 = F8.dequant_pool(db.v8.cpu().numpy(), db.v_scale.cpu().numpy())
-        ref8 = A8.attend_decode(b.q_decode, K8, V8, b.block_table, b.kv_lens, b.scale, w.num_kv_heads,
-                                requests=reqs8, first_row=b.num_prefill)
+        # only the sampled requests' blocks are copied back and decoded (block table remapped onto them)
+        rows8 = [b.num_prefill + r for r in reqs8]
+        npg = [-(-int(b.kv_lens[r]) // 16) for r in rows8]
+        blocks = np.unique(np.concatenate([b.block_table[r, :n] for r, n in zip(rows8, npg)]))
+        remap = {int(x): i for i, x in enumerate(blocks)}
+        bt8 = np.zeros((len(rows8), max(npg)), dtype=np.int32)
+        for i, (r, n) in enumerate(zip(rows8, npg)):
+            bt8[i, :n] = [remap[int(x)] for x in b.block_table[r, :n]]
+        idx = torch.from_numpy(blocks.astype(np.int64)).to(db.k8.device)
+        K8 = F8.dequant_pool(db.k8[idx].cpu().numpy(), db.k_scale.cpu().numpy())
+        V8 = F8.dequant_pool(db.v8[idx].cpu().numpy(), db.v_scale.cpu().numpy())
+        ref8 = A8.attend_decode(b.q_decode[reqs8], K8, V8, bt8, np.asarray([int(b.kv_lens[r]) for r in rows8]),
+                                b.scale, w.num_kv_heads, first_row=0)
         got8 = db.o_dec.float().cpu().numpy()[reqs8]
         fp8_arm["parity_sample"] = {"requests": reqs8, "max_abs": float(np.abs(got8 - ref8).max()),
                                     "mean_abs": float(np.abs(got8 - ref8).mean())}

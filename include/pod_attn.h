@@ -88,7 +88,8 @@ enum {
                                           decode (the MMA and TMA warps too; rings 2 / 3 deep) */
 #define POD_FLAG_PREFILL_SPLIT_UNLIMITED 128u /* ablation: the prefill KV split fills every CTA slot even
                                                  when a short prefill (<= 1536 tokens) shares the batch
-                                                 with decode work (the plan rule's co-located limit off) */
+                                                 with decode work (the plan rule's co-located limit off,
+                                                 which otherwise counts one prefill slot per SM) */
 
 typedef struct pod_attn_config {
   int32_t num_q_heads;      /* Hq, 1..4096 */
@@ -160,9 +161,10 @@ typedef struct pod_attn_plan_info {
  *    B200 tensor FLOP/s per HBM byte/s), tot = cost_pre + cost_dec,
  *    n_p = floor((2 k cost_pre + tot) / (2 tot)) clamped to [1, k-1] (k = 1:
  *    n_p = 1), and n_p = k when 2 cost_pre >= tot; p:d = n_p : k - n_p reduced.
- *  - Prefill KV split: h_p = #{t in [0,k): t mod (p+d) < p}; limited = there
- *    are decodes and sum_i P_i <= 1536 and POD_FLAG_PREFILL_SPLIT_UNLIMITED is
- *    off; slots = num_sms * (limited ? max(h_p, 1) : k).  With n0 base items:
+ *  - Prefill KV split: limited = there are decodes and sum_i P_i <= 1536 and
+ *    POD_FLAG_PREFILL_SPLIT_UNLIMITED is off; slots = num_sms if limited (one
+ *    prefill slot per SM: the SM's other CTA stays for decode), else
+ *    num_sms * k.  With n0 base items:
  *    if max_prefill_splits == 1 or n0 == 0 or n0 >= slots, nothing is split;
  *    else tau = max(8, ceil(sum n / slots)) and an item of n tiles gets
  *    S = min(smax, max(1, floor(n / tau))) pieces (smax = max_prefill_splits

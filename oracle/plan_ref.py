@@ -27,9 +27,11 @@ Rule
   Prefill KV split (after the ratio below; FlashInfer PR "Limit kv split when
     prefill tokens <= 1536": the prefill's split count leaves room for the
     decode CTAs co-located on the same SMs while the prefill is short):
-    h_p = number of t in 0 .. k-1 with t mod (p+d) < p (prefill-home CTAs
-    per SM); limited = (B > 0 and sum_i P_i <= 1536 and the unlimited
-    ablation is off); slots = num_sms * (max(h_p, 1) if limited else k);
+    limited = (B > 0 and sum_i P_i <= 1536 and the unlimited ablation is
+    off); slots = num_sms if limited (one prefill slot per SM: the SM's
+    other CTA, decode-home or a second prefill-home one, stays for decode;
+    measured on B200, a second prefill CTA adds only ~15% to an SM's prefill
+    throughput) else num_sms * k;
     n0 = number of base items.  If prefill_splits == 1, or n0 == 0, or
     n0 >= slots: every item has S = 1 piece.  Otherwise W = sum of n over the
     base items, tau = max(8, ceil(W / slots)) and an item of n tiles gets
@@ -244,9 +246,8 @@ def plan_ref_batched(num_q_heads: int, num_kv_heads: int, head_dim: int, num_sms
             p_, d_ = p_ // gg, d_ // gg
 
     # prefill KV split
-    h_p = sum(1 for t in range(k) if (p_ + d_) > 0 and t % (p_ + d_) < p_)
     limited = B > 0 and sum(pre_qo) <= SPLIT_LIMIT_TOKENS and not split_unlimited
-    slots = num_sms * (max(h_p, 1) if limited else k)
+    slots = num_sms if limited else num_sms * k
     tiles = [_ceil(kv_end, BN) for (_, _, kv_end, _) in pre]
     n0 = len(pre)
     if prefill_splits == 1 or n0 == 0 or n0 >= slots:

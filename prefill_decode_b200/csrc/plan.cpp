@@ -211,13 +211,11 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
   pl->ratio_d = rd;
 
   // ---- prefill KV split: fill the prefill CTA slots when the base items leave some empty;
-  // a short prefill (<= 1536 tokens) next to decode work counts only its prefill-home CTAs
+  // a short prefill (<= 1536 tokens) next to decode work counts one slot per SM (the SM's
+  // other CTA stays for decode; a second prefill CTA on an SM adds little throughput)
   {
-    int32_t hp = 0;
-    for (int32_t t = 0; t < k; ++t)
-      if (rp + rd > 0 && t % (rp + rd) < rp) ++hp;
     const bool limited = B > 0 && sumP <= kSplitLimitTokens && !(cfg->flags & POD_FLAG_PREFILL_SPLIT_UNLIMITED);
-    const int64_t slots = (int64_t)num_sms * (limited ? std::max<int32_t>(hp, 1) : k);
+    const int64_t slots = limited ? (int64_t)num_sms : (int64_t)num_sms * k;
     const int64_t n0 = (int64_t)base.size();
     std::vector<int32_t> nsplit(base.size(), 1);
     if (cfg->max_prefill_splits != 1 && n0 > 0 && n0 < slots) {

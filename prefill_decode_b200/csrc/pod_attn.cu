@@ -753,9 +753,11 @@ __device__ void merge_row_warp(const PodParams& p, int midx) {
 //  * keys: score row r of the 16-row tile is key sigma(r) of the page, chosen so
 //    that after the movmatrix transpose the P^T fragment of lane (n, q) holds
 //    keys sigma(2q), sigma(2q+1), sigma(2q+8), sigma(2q+9) = the 4q..4q+3 block,
-//    which is what one 32-bit load per key row of V provides;
-//  * in O^T = V^T P^T, the 16 output rows of M-tile 2p + t are d values
-//    32p + 4g + 2t (rows g) and 32p + 4g + 2t + 1 (rows g + 8).
+//    so the lane reads exactly four key rows of V;
+//  * in O^T = V^T P^T, lane (g, q) owns the d/8 consecutive d values starting at
+//    (d/8) g: M-tile mt holds d = (d/8) g + 2 mt (rows g) and + 1 (rows g + 8),
+//    so one 16-byte (8-byte at d = 64) load per key row feeds every M-tile, and
+//    each head's outputs of a lane are contiguous.
 // sigma(r) = 4 q' + e + 2 (hi ^ (q' >> 1)) with q' = (r & 7) >> 1, e = r & 1,
 // hi = r >> 3: the 2-key blocks of lanes q >= 2 are swapped, which spreads the
 // four key rows one V load instruction touches over distinct swizzle phases.
@@ -923,42 +925,64 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
       const float s2 = key_hi < valid ? c[2] * sl2 : -INFINITY;
       const float s3 = key_hi < valid ? c[3] * sl2 : -INFINITY;
       float tA = fmaxf(s0, s2), tB = fmaxf(s1, s3);
+      // the running max is kept stale until a score beats it by more than 2^8 (any base gives the same
+      // softmax; exponentials stay <= 2^8): only then reduce the page max across lanes and rescale
+      if (__any_sync(0xffffffffu, tA > mA + 8.f || tB > mB + 8.f)) {
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        tA = fmaxf(tA, __shfl_xor_sync(0xffffffffu, tA, o));
-        tB = fmaxf(tB, __shfl_xor_sync(0xffffffffu, tB, o));
-      }
-      const float nA = fmaxf(mA, tA), nB = fmaxf(mB, tB);
-      const float alA = ex2(mA - nA), alB = ex2(mB - nB);
-      mA = nA;
-      mB = nB;
-      const float e0 = ex2(s0 - nA), e1 = ex2(s1 - nB), e2 = ex2(s2 - nA), e3 = ex2(s3 - nB);
-      lA = lA * alA + e0 + e2;
-      lB = lB * alB + e1 + e3;
+        for (int o = 4; o < 32; o <<= 1) {
+          tA = fmaxf(tA, __shfl_xor_sync(0xffffffffu, tA, o));
+          tB = fmaxf(tB, __shfl_xor_sync(0xffffffffu, tB, o));
+        }
+        const float nA = fmaxf(mA, tA), nB = fmaxf(mB, tB);
+        const float alA = ex2(mA - nA), alB = ex2(mB - nB);
+        mA = nA;
+        mB = nB;
+        lA *= alA;
+        lB *= alB;
 #pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {
-        acc[mt][0] *= alA;
-        acc[mt][1] *= alB;
-        acc[mt][2] *= alA;
-        acc[mt][3] *= alB;
+        for (int mt = 0; mt < D / 16; ++mt) {
+          acc[mt][0] *= alA;
+          acc[mt][1] *= alB;
+          acc[mt][2] *= alA;
+          acc[mt][3] *= alB;
+        }
       }
+      const float e0 = ex2(s0 - mA), e1 = ex2(s1 - mB), e2 = ex2(s2 - mA), e3 = ex2(s3 - mB);
+      lA += e0 + e2;
+      lB += e1 + e3;
       if constexpr (KV8) {
         const uint32_t pb0 = movmatrix_t(pack_f16(e0, e1));   // score rows 0..7
         const uint32_t pb1 = movmatrix_t(pack_f16(e2, e3));   // score rows 8..15
         // this lane's V key rows sigma(2q), sigma(2q+1), sigma(2q+8), sigma(2q+9)
         const int rot = 2 * (q4 >> 1);
         const int ra = 4 * q4 + rot, rb = ra + 1, rc = 4 * q4 + (rot ^ 2), rd = rc + 1;
+        // lane (gq, q) owns d = (D/8) gq .. +D/8-1: M-tile mt holds d = (D/8) gq + 2 mt (rows gq) and +1
+        constexpr int W = D / 32;                  // 32-bit words of a lane's d range per key row
+        uint32_t wa[W], wb[W], wc[W], wd[W];
+        {
+          const int col = (D / 8) * gq;
+          if constexpr (W == 4) {
+            const uint4 a4 = lds_u128(vb_u + page8_off<D>(ra, col)), b4 = lds_u128(vb_u + page8_off<D>(rb, col));
+            const uint4 c4 = lds_u128(vb_u + page8_off<D>(rc, col)), d4 = lds_u128(vb_u + page8_off<D>(rd, col));
+            wa[0] = a4.x; wa[1] = a4.y; wa[2] = a4.z; wa[3] = a4.w;
+            wb[0] = b4.x; wb[1] = b4.y; wb[2] = b4.z; wb[3] = b4.w;
+            wc[0] = c4.x; wc[1] = c4.y; wc[2] = c4.z; wc[3] = c4.w;
+            wd[0] = d4.x; wd[1] = d4.y; wd[2] = d4.z; wd[3] = d4.w;
+          } else {
+            const uint2 a2 = lds_u64(vb_u + page8_off<D>(ra, col)), b2 = lds_u64(vb_u + page8_off<D>(rb, col));
+            const uint2 c2v = lds_u64(vb_u + page8_off<D>(rc, col)), d2 = lds_u64(vb_u + page8_off<D>(rd, col));
+            wa[0] = a2.x; wa[1] = a2.y; wb[0] = b2.x; wb[1] = b2.y;
+            wc[0] = c2v.x; wc[1] = c2v.y; wd[0] = d2.x; wd[1] = d2.y;
+          }
+        }
 #pragma unroll
-        for (int pg = 0; pg < D / 32; ++pg) {
-          const int col = 32 * pg + 4 * gq;
-          const uint32_t va = lds_u32(vb_u + page8_off<D>(ra, col)), vb = lds_u32(vb_u + page8_off<D>(rb, col));
-          const uint32_t vc = lds_u32(vb_u + page8_off<D>(rc, col)), vd = lds_u32(vb_u + page8_off<D>(rd, col));
-          // byte pairs (key a, key b) for d = col + 0/1 and col + 2/3
-          const uint32_t ab01 = __byte_perm(va, vb, 0x5140), ab23 = __byte_perm(va, vb, 0x7362);
-          const uint32_t cd01 = __byte_perm(vc, vd, 0x5140), cd23 = __byte_perm(vc, vd, 0x7362);
-          mma_16816_f16(acc[2 * pg], lo16_e4m3_to_f16x2(ab01), hi16_e4m3_to_f16x2(ab01), lo16_e4m3_to_f16x2(cd01),
+        for (int w = 0; w < W; ++w) {
+          // byte pairs (key a, key b) for d = 4w + 0/1 (M-tile 2w) and 4w + 2/3 (M-tile 2w + 1)
+          const uint32_t ab01 = __byte_perm(wa[w], wb[w], 0x5140), ab23 = __byte_perm(wa[w], wb[w], 0x7362);
+          const uint32_t cd01 = __byte_perm(wc[w], wd[w], 0x5140), cd23 = __byte_perm(wc[w], wd[w], 0x7362);
+          mma_16816_f16(acc[2 * w], lo16_e4m3_to_f16x2(ab01), hi16_e4m3_to_f16x2(ab01), lo16_e4m3_to_f16x2(cd01),
                         hi16_e4m3_to_f16x2(cd01), pb0, pb1);
-          mma_16816_f16(acc[2 * pg + 1], lo16_e4m3_to_f16x2(ab23), hi16_e4m3_to_f16x2(ab23),
+          mma_16816_f16(acc[2 * w + 1], lo16_e4m3_to_f16x2(ab23), hi16_e4m3_to_f16x2(ab23),
                         lo16_e4m3_to_f16x2(cd23), hi16_e4m3_to_f16x2(cd23), pb0, pb1);
         }
       } else {
@@ -1011,18 +1035,19 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
     if (part < 0) {
       __nv_bfloat16* ob = p.o_dec + ((size_t)r * p.Hq + kvh * g) * D;
       if constexpr (KV8) {
-        // M-tile 2pg + t holds d = 32 pg + 4 gq + 2t (+1 in rows gq + 8): four consecutive d per head
+        // M-tile mt holds d = (D/8) gq + 2 mt (+1 in rows gq + 8): D/8 consecutive d per head
 #pragma unroll
-        for (int pg = 0; pg < D / 32; ++pg) {
-          const int dd = 32 * pg + 4 * gq;
+        for (int v = 0; v < D / 64; ++v) {
+          const int dd = (D / 8) * gq + 8 * v;
+          const int m0 = 4 * v;
           if (hA < g)
-            *reinterpret_cast<uint2*>(ob + hA * D + dd) =
-                make_uint2(pack_bf16(acc[2 * pg][0] * iA, acc[2 * pg][2] * iA),
-                           pack_bf16(acc[2 * pg + 1][0] * iA, acc[2 * pg + 1][2] * iA));
+            *reinterpret_cast<uint4*>(ob + hA * D + dd) =
+                make_uint4(pack_bf16(acc[m0][0] * iA, acc[m0][2] * iA), pack_bf16(acc[m0 + 1][0] * iA, acc[m0 + 1][2] * iA),
+                           pack_bf16(acc[m0 + 2][0] * iA, acc[m0 + 2][2] * iA), pack_bf16(acc[m0 + 3][0] * iA, acc[m0 + 3][2] * iA));
           if (hB < g)
-            *reinterpret_cast<uint2*>(ob + hB * D + dd) =
-                make_uint2(pack_bf16(acc[2 * pg][1] * iB, acc[2 * pg][3] * iB),
-                           pack_bf16(acc[2 * pg + 1][1] * iB, acc[2 * pg + 1][3] * iB));
+            *reinterpret_cast<uint4*>(ob + hB * D + dd) =
+                make_uint4(pack_bf16(acc[m0][1] * iB, acc[m0][3] * iB), pack_bf16(acc[m0 + 1][1] * iB, acc[m0 + 1][3] * iB),
+                           pack_bf16(acc[m0 + 2][1] * iB, acc[m0 + 2][3] * iB), pack_bf16(acc[m0 + 3][1] * iB, acc[m0 + 3][3] * iB));
         }
       } else {
         const int d_lo = gq;
@@ -1043,14 +1068,15 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
       float* po = p.part_o + (size_t)part * g * D;
       if constexpr (KV8) {
 #pragma unroll
-        for (int pg = 0; pg < D / 32; ++pg) {
-          const int dd = 32 * pg + 4 * gq;
+        for (int v = 0; v < D / 32; ++v) {
+          const int dd = (D / 8) * gq + 4 * v;
+          const int m0 = 2 * v;
           if (hA < g)
-            *reinterpret_cast<float4*>(po + hA * D + dd) = make_float4(
-                acc[2 * pg][0] * iA, acc[2 * pg][2] * iA, acc[2 * pg + 1][0] * iA, acc[2 * pg + 1][2] * iA);
+            *reinterpret_cast<float4*>(po + hA * D + dd) =
+                make_float4(acc[m0][0] * iA, acc[m0][2] * iA, acc[m0 + 1][0] * iA, acc[m0 + 1][2] * iA);
           if (hB < g)
-            *reinterpret_cast<float4*>(po + hB * D + dd) = make_float4(
-                acc[2 * pg][1] * iB, acc[2 * pg][3] * iB, acc[2 * pg + 1][1] * iB, acc[2 * pg + 1][3] * iB);
+            *reinterpret_cast<float4*>(po + hB * D + dd) =
+                make_float4(acc[m0][1] * iB, acc[m0][3] * iB, acc[m0 + 1][1] * iB, acc[m0 + 1][3] * iB);
         }
       } else {
         const int d_lo = gq;

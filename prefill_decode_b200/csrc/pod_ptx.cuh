@@ -266,9 +266,9 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
 }
 __device__ __forceinline__ uint32_t lo16_e4m3_to_f16x2(uint32_t w) { return e4m3x2_to_f16x2((uint16_t)(w & 0xFFFFu)); }
 __device__ __forceinline__ uint32_t hi16_e4m3_to_f16x2(uint32_t w) { return e4m3x2_to_f16x2((uint16_t)(w >> 16)); }
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
   return v;
 }
 __device__ __forceinline__ uint4 lds_u128(uint32_t addr) {

@@ -410,3 +410,15 @@ def test_planted_split_mistakes_fail_the_piece_invariants():
         bad.prefill_items[0, col] += delta
         with pytest.raises(AssertionError):
             check_prefill_pieces(bad, 1, [64], [1664])
+
+
+def test_prefill_split_limited_counts_one_slot_per_sm():
+    """With every CTA prefill-home (ratio 1:0) a short prefill beside decode work still counts one prefill
+    slot per SM: the Llama-3-8B mix's 128 items are not cut (a second prefill CTA on an SM would only queue
+    behind the first); without the limit they are cut for all 296 CTA slots."""
+    w = synth.llama3_8b_mix()
+    forced = _plan(w, ratio_p=1, ratio_d=0)
+    assert (forced.ratio_p, forced.ratio_d) == (1, 0) and forced.num_prefill_partials == 0
+    assert _plan(w, ratio_p=1, ratio_d=0, split_unlimited=True).num_prefill_partials == 256
+    one = _plan(w, ctas_per_sm=1, split_unlimited=True)      # one CTA per SM: 148 slots either way
+    assert one.num_prefill_partials == _plan(w, ctas_per_sm=1).num_prefill_partials == 0
