@@ -47,15 +47,26 @@ KERNEL_SOURCES = ["prefill_decode_b200/csrc/pod_attn.cu", "prefill_decode_b200/c
 HOST_SIDE_MARKER = b"// =========================================================== host side (ABI)"
 
 
+def _code_only(data: bytes) -> bytes:
+    """C++ source without comments and with whitespace runs collapsed, so that an
+    edit to a comment does not count as a change of the device code."""
+    import re
+    text = data.decode("utf-8", "replace")
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return re.sub(r"\s+", " ", text).strip().encode()
+
+
 def kernel_source_sha(root: str = ROOT) -> str:
-    """Hash of the device code: the kernel sources, with the host-side ABI part
-    of the .cu file (launch plumbing, tensor-map encoding) left out."""
+    """Hash of the device code: the kernel sources without comments, with the
+    host-side ABI part of the .cu file (launch plumbing, tensor-map encoding)
+    left out."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         with open(os.path.join(root, f), "rb") as fh:
             data = fh.read()
         i = data.find(HOST_SIDE_MARKER)
-        h.update(data if i < 0 else data[:i])
+        h.update(_code_only(data if i < 0 else data[:i]))
     return h.hexdigest()[:16]
 
 

@@ -11,15 +11,20 @@
 //     roles per SM in software");
 //   * decode runs in single-warp virtual blocks ("Balance shared memory and
 //     threadblock count") with small tensor-core tiles ("Shrink decode tiles");
-//   * KV is split for decode parallelism, capped by the plan ("Cap prefill
-//     splitting"), and the splits are merged by log-sum-exp (PAT record).
+//   * KV is split for decode parallelism, and for the prefill when its items
+//     leave CTA slots empty, capped by the plan ("Cap prefill splitting"; the
+//     FlashInfer PR "Limit kv split when prefill tokens <= 1536" keeps room
+//     for co-located decode CTAs); splits are merged by log-sum-exp (PAT
+//     record) by whoever finishes a row's last split.
 // B200 re-design (prior art, not the blueprint): CTAs are persistent -- the
 // ticket fixes a CTA's home role, the CTA drains that role's queue and then
 // steals from the other, so no CTA ever waits on another.  Prefill tiles are
 // 128 x 64 tcgen05 MMAs: S = Q K^T with Q held in TMEM, O += P V with P staged
 // in shared memory, both accumulated in TMEM; K and V arrive by TMA with
 // 128-byte swizzle straight from the 16-token pages.  Decode warps stage pages
-// with TMA into a per-warp ring and use m16n8k16 MMAs with keys as rows.
+// with TMA into a per-warp ring and use m16n8k16 MMAs with keys as rows, on
+// bf16 pages or on e4m3 pages converted to f16 in registers (the FP8 cache of
+// the blog post "Prefill vs. Decode GPU Utilization Imbalance").
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -88,7 +93,7 @@ struct alignas(64) PodParams {
 };
 
 constexpr int kThreads = 192;        // warps 0-3: softmax (prefill) / decode units; warp 4: MMA; warp 5: TMA
-                                     // (in decode, warps 4 and 5 idle, or decode too when decode_warps == 6)
+                                     // (in decode, warps 4 and 5 decode too, or idle with decode_warps == 4)
 constexpr int kMmaWarp = 4;
 constexpr int kTmaWarp = 5;
 constexpr int kAllWarps = kThreads / 32;

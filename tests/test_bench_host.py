@@ -48,7 +48,9 @@ def test_kernel_hash_ignores_the_host_side_part(tmp_path):
     data = cu.read_bytes()
     i = data.find(bench.HOST_SIDE_MARKER)
     assert i > 0
-    cu.write_bytes(data[:i] + b"// a device-side edit\n" + data[i:])
+    cu.write_bytes(data[:i] + b"// a comment-only device-side edit\n/* and a block comment */\n" + data[i:])
+    assert bench.kernel_source_sha(str(root)) == base
+    cu.write_bytes(data[:i] + b"__device__ int pod_hash_probe;\n" + data[i:])
     assert bench.kernel_source_sha(str(root)) != base
 
 
