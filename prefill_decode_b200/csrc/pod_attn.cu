@@ -102,9 +102,10 @@ constexpr int kAllWarps = kThreads / 32;
 enum : int {
   kBarQ = 0,        // Q rows of the item stored into TMEM                      count 4 (softmax warps)
   kBarKFull = 1,    // [3] K tile landed (TMA)                                  count 1 + tx
-  kBarKEmpty = 4,   // [3] K slot free again: its S MMA finished (commit)       count 1
+  kBarSFull = 4,    // [3] S_t ready in TMEM, [t % 3] (commit); K slot t % 3   count 1
+                    //     is free again (one commit serves both: ~200 cycles each)
   kBarVFull = 7,    // [2] V tile landed (TMA)                                  count 1 + tx
-  kBarSFull = 9,    // S tile ready in TMEM (commit)                            count 1
+  // 9: unused
   kBarSFree = 10,   // softmax has read S out of TMEM                           count 4 (softmax warps)
   kBarPFull = 11,   // [2] P tile t stored in shared-memory buffer t&1          count 4 (softmax warps)
   kBarODone = 13,   // [2] P.V MMA of tile t finished: P buffer and V slot t&1  count 1
@@ -112,12 +113,12 @@ enum : int {
   kBarOFinal = 15,  // last P.V MMA of an item finished (commit)                count 1
   kBarDecode = 16,  // [decode warps * ring depth] decode page rings            count 1 + tx
 };
-// Parity waits are only sound when the waiter knows the barrier is at most one
-// phase away from the one it waits for.  For key tile t (counted over the
-// CTA's lifetime): S_{t+1} is issued only after the softmax has read S_t
-// (s_free), and the softmax reads S_{t+1} only after S_t, so s_full and s_free
-// alternate; K_{t+3} is loaded into slot t%3 after S_t finished (k_empty) and
-// S_{t+3} needs it; P_t goes into buffer t&1 only after P.V_{t-2} finished and
+// Parity waits are only sound when the waiter for completion k of a barrier
+// knows that completion k + 1 cannot have happened yet.  For key tile t
+// (counted over the CTA's lifetime): s_full[t % 3] completes once per three
+// tiles; the softmax waits on it for S_t, and S_{t+3} needs the softmax to have
+// read S_{t+2} (s_free); the TMA warp waits on it before K_{t+3} goes into slot
+// t % 3, and S_{t+3} needs that K tile; P_t goes into buffer t&1 only after P.V_{t-2} finished and
 // P.V_t needs P_t, so p_full is at most one phase ahead per buffer; o_done[t&1]
 // is waited on by the TMA warp (before V_{t+2} goes into slot t&1) and by the
 // softmax (tiles t+1 and t+2, before it rescales O or reuses the P buffer),
@@ -290,7 +291,7 @@ __device__ bool prefill_tma(const PodParams& p, const PreItem& it, uint8_t* smem
     const int rk = more_k ? tile_page_row(p, pw, j0 + j + CF::kKSlots, kvh, kv_end, lane) : 0;
     const int rv = tile_page_row(p, pw, j0 + j + CF::kVSlots, kvh, kv_end, lane);
     if (more_k) {                // K first: S_{t+3} is issued well before P.V_{t+2}
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarKEmpty + t % 3], (t / 3) & 1u, kWaitLimitNs))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + t % 3], (t / 3) & 1u, kWaitLimitNs))) return false;
       issue_tile<D>(&p.tm_k, sm.k(t + CF::kKSlots), &bars[kBarKFull + t % 3], rk, lane);
     }
     if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarODone + (t & 1u)], (t >> 1) & 1u, kWaitLimitNs))) return false;
@@ -302,8 +303,9 @@ __device__ bool prefill_tma(const PodParams& p, const PreItem& it, uint8_t* smem
 // MMA warp of one prefill item (lane 0 issues): S_t = Q K_t^T into TMEM with Q
 // read from TMEM (stored there by the softmax warps), issued as soon as the
 // softmax has read S_{t-1} out; O += P_t V_t with P_t read from shared memory.
-// Commits free the K slot right after S_t and the V slot and the P buffer
-// after P.V_t.
+// One commit after S_t (s_full: S ready, K slot free) and one after P.V_t
+// (o_done: V slot and P buffer free); a commit holds the issuing thread ~200
+// cycles, so each serves every consumer it can.
 template <int D>
 __device__ bool prefill_mma(const PodParams& p, const PreItem& it, uint8_t* smem, uint64_t* bars, uint32_t tmem,
                             uint32_t t0, uint32_t nq) {
@@ -327,8 +329,7 @@ __device__ bool prefill_mma(const PodParams& p, const PreItem& it, uint8_t* smem
       const uint32_t boff = ((kk >> 2) * (kBN * 128) + (kk & 3) * 32) >> 4;
       umma_bf16_tmem_a(tmem + kTmemS, tmem + kTmemQ + kk * 8, dk + boff, idesc_s, kk > 0 ? 1u : 0u);
     }
-    umma_commit(&bars[kBarSFull]);
-    umma_commit(&bars[kBarKEmpty + t % 3]);
+    umma_commit(&bars[kBarSFull + t % 3]);
   };
 
   {                              // S of the first tile, once Q is in TMEM
@@ -435,7 +436,7 @@ __device__ bool prefill_softmax(const PodParams& p, const PreItem& it, int item,
   for (int jj = 0; jj < nkb; ++jj) {
     const int j = j0 + jj;       // absolute key tile
     const uint32_t t = t0 + jj;
-    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull], t & 1u, kWaitLimitNs))) return false;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull + t % 3], (t / 3) & 1u, kWaitLimitNs))) return false;
     tc_fence_after();
     float s[kBN];
     tmem_ld32(tmem + t_lane + kTmemS, s);
@@ -620,26 +621,31 @@ __device__ bool prefill_softmax(const PodParams& p, const PreItem& it, int item,
 // O^T[d x 8] += V_page^T . P^T.  Pages arrive by TMA into a kNS-deep ring.
 // The block ids of an item's pages are read 32 at a time, one per lane, a
 // window ahead of use, so refilling a ring slot never waits on a global load.
+// Called by the whole warp: lane 0 expects the stage's bytes, then lanes 0 and 1
+// issue the K and the V box of the page in one TMA instruction (a TMA
+// instruction holds its warp ~130 cycles plus ~50 per box, so one instruction of
+// two boxes costs less than two of one).
 template <int D, int NS, bool KV8>
 __device__ __forceinline__ void decode_issue_page(const PodParams& p, uint8_t* ring, uint64_t* wbars, uint32_t seq,
-                                                  int blk, int kvh) {
+                                                  int blk, int kvh, int lane) {
   using CF = Cfg<D>;
   constexpr int kStage = KV8 ? CF::kDecStage8 : CF::kDecStage;
   constexpr int kPageB = KV8 ? CF::kPageBytes8 : CF::kPageBytes;
   const int s = seq % NS;
-  uint8_t* kbuf = ring + s * kStage;
+  uint8_t* dst = ring + s * kStage + (lane == 1 ? kPageB : 0);
   uint64_t* bar = &wbars[s];
-  mbar_arrive_expect_tx(bar, kStage);
-  const int row = KV8 ? kv_row8(p, blk, kvh) : kv_row(p, blk, kvh);
-  if constexpr (KV8) {
-    // one box per e4m3 page of K and of V: 16 rows of d bytes (128-byte swizzle at d = 128)
-    tma_load_2d(kbuf, &p.tm_k8, bar, 0, row);
-    tma_load_2d(kbuf + kPageB, &p.tm_v8, bar, 0, row);
-  } else {
-    // one box per page of K and of V: both 64-element halves of 16 rows land as
-    // [half][16 rows][128 B], the layout two 2D boxes would give
-    tma_load_3d(kbuf, &p.tm_kp, bar, 0, row, 0);
-    tma_load_3d(kbuf + kPageB, &p.tm_vp, bar, 0, row, 0);
+  if (lane == 0) mbar_arrive_expect_tx(bar, kStage);
+  if (lane < 2) {
+    const int row = KV8 ? kv_row8(p, blk, kvh) : kv_row(p, blk, kvh);
+    if constexpr (KV8) {
+      // one box per e4m3 page of K (lane 0) and of V (lane 1): 16 rows of d bytes
+      // (128-byte swizzle at d = 128)
+      tma_load_2d(dst, lane == 0 ? &p.tm_k8 : &p.tm_v8, bar, 0, row);
+    } else {
+      // one box per page of K (lane 0) and of V (lane 1): both 64-element halves of
+      // 16 rows land as [half][16 rows][128 B], the layout two 2D boxes would give
+      tma_load_3d(dst, lane == 0 ? &p.tm_kp : &p.tm_vp, bar, 0, row, 0);
+    }
   }
 }
 
@@ -811,7 +817,7 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
       const int pre = np < NS ? np : NS;
       for (int j = 0; j < pre; ++j) {
         const int blk = __shfl_sync(0xffffffffu, bt_cur, j);
-        if (lane == 0) decode_issue_page<D, NS, KV8>(p, ring, wbars, seq + j, blk, kvh);
+        decode_issue_page<D, NS, KV8>(p, ring, wbars, seq + j, blk, kvh, lane);
       }
     }
     if (lane == 0) {
@@ -1011,7 +1017,7 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         }
         const int blk = __shfl_sync(0xffffffffu, bt_cur, jn & 31);
         __syncwarp();
-        if (lane == 0) decode_issue_page<D, NS, KV8>(p, ring, wbars, sq + NS, blk, kvh);
+        decode_issue_page<D, NS, KV8>(p, ring, wbars, sq + NS, blk, kvh, lane);
       }
     }
     if (!ok) {

@@ -72,7 +72,7 @@ def _rising_decode_batch():
         for kvh in range(2):
             for j in range(L):
                 blk = int(b.block_table[row, j // PAGE])
-                b.k_pool[blk, kvh, j % PAGE, 0] = _bf16(60.0 * j / L)
+                b.k_pool[blk, kvh, j % PAGE, 0] = _bf16(60.0 * j / L).reshape(-1)[0]
     b.q_decode[:, :, 0] = _bf16(16.0)
     return b
 
