@@ -567,45 +567,75 @@ __device__ bool prefill_softmax(const PodParams& p, const PreItem& it, int item,
   int last = 0;
   if (lane == 0) last = atomicAdd(&p.pmerge_cnt[kWarpsPerCta * midx + warp], 1) == pm.y - 1;
   last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last || q >= P) return true;
+  if (!last) return true;
   __threadfence();
-  // O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s (log2 domain);
-  // the other pieces' partials were written by other CTAs of this launch: read them through L2
+  // O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s (log2 domain), over the warp's 32
+  // rows; the other pieces' partials were written by other CTAs of this launch: read them through L2.
+  // Each thread first turns its row's log-sum-exps into normalised weights (one batch of loads) and parks
+  // them in this warp's part of the P buffers (free: every P.V MMA of the item has finished); then it reads
+  // its row's partials two pieces per batch of loads, so a row costs about 1 + (d/32) * pieces/2 round trips
+  // (the epilogue of a split item took up to 30 us when every load waited for the one before).
   const int first = pm.x, S = pm.y;
-  const float* lse = p.ppart_lse + (size_t)first * kBM + row;
-  float M = -INFINITY;
-  for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(lse + (size_t)sp * kBM));
-  float den = 0.f;
-  for (int sp = 0; sp < S; ++sp) den += ex2(__ldcg(lse + (size_t)sp * kBM) - M);
-  const float dinv = 1.f / den;
+  const int row0 = warp * 32;
+  float* wtab = reinterpret_cast<float*>(smem + Cfg<D>::kOffP) + warp * (kMaxPrefillPieces * 32);
+  {
+    // the (at most 16) log-sum-exps of lane's row in one batch of loads, then max, weights, sum
+    const float* lse = p.ppart_lse + (size_t)first * kBM + row0 + lane;
+    float M = -INFINITY;
+#pragma unroll
+    for (int sp = 0; sp < kMaxPrefillPieces; ++sp) {
+      if (sp < S) {
+        const float x = __ldcg(lse + (size_t)sp * kBM);
+        wtab[sp * 32 + lane] = x;
+        M = fmaxf(M, x);
+      }
+    }
+    float den = 0.f;
+#pragma unroll 1
+    for (int sp = 0; sp < S; ++sp) {
+      const float e = ex2(wtab[sp * 32 + lane] - M);
+      wtab[sp * 32 + lane] = e;
+      den += e;
+    }
+    const float dinv = 1.f / den;   // rows past the chunk (never written) give garbage weights, never used
+#pragma unroll 1
+    for (int sp = 0; sp < S; ++sp) wtab[sp * 32 + lane] *= dinv;
+  }
+  __syncwarp();
+  if (q >= P) return true;
 #pragma unroll 1
   for (int c = 0; c < D / 32; ++c) {
     float acc[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) acc[k] = 0.f;
 #pragma unroll 1
-    for (int sp = 0; sp < S; ++sp) {
-      const float w = ex2(__ldcg(lse + (size_t)sp * kBM) - M);
-      const float4* src = reinterpret_cast<const float4*>(p.ppart_o + ((size_t)(first + sp) * kBM + row) * D + c * 32);
-      float4 v[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = __ldcg(src + k);
+    for (int sp = 0; sp < S; sp += 2) {
+      const int sp1 = sp + 1 < S ? sp + 1 : sp;   // a valid address either way; its weight is 0 then
+      const float wa = wtab[sp * 32 + lane], wb = sp + 1 < S ? wtab[sp1 * 32 + lane] : 0.f;
+      const float4* pa = reinterpret_cast<const float4*>(p.ppart_o + ((size_t)(first + sp) * kBM + row) * D + c * 32);
+      const float4* pb = reinterpret_cast<const float4*>(p.ppart_o + ((size_t)(first + sp1) * kBM + row) * D + c * 32);
+      float4 va[8], vb[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        acc[4 * k] += w * v[k].x;
-        acc[4 * k + 1] += w * v[k].y;
-        acc[4 * k + 2] += w * v[k].z;
-        acc[4 * k + 3] += w * v[k].w;
+        va[k] = __ldcg(pa + k);
+        vb[k] = __ldcg(pb + k);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        acc[4 * k] += wa * va[k].x + wb * vb[k].x;
+        acc[4 * k + 1] += wa * va[k].y + wb * vb[k].y;
+        acc[4 * k + 2] += wa * va[k].z + wb * vb[k].z;
+        acc[4 * k + 3] += wa * va[k].w + wb * vb[k].w;
       }
     }
     uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       uint4 v;
-      v.x = pack_bf16(acc[k * 8 + 0] * dinv, acc[k * 8 + 1] * dinv);
-      v.y = pack_bf16(acc[k * 8 + 2] * dinv, acc[k * 8 + 3] * dinv);
-      v.z = pack_bf16(acc[k * 8 + 4] * dinv, acc[k * 8 + 5] * dinv);
-      v.w = pack_bf16(acc[k * 8 + 6] * dinv, acc[k * 8 + 7] * dinv);
+      v.x = pack_bf16(acc[k * 8 + 0], acc[k * 8 + 1]);
+      v.y = pack_bf16(acc[k * 8 + 2], acc[k * 8 + 3]);
+      v.z = pack_bf16(acc[k * 8 + 4], acc[k * 8 + 5]);
+      v.w = pack_bf16(acc[k * 8 + 6], acc[k * 8 + 7]);
       dst[k] = v;
     }
   }
