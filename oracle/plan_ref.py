@@ -29,9 +29,8 @@ Rule
     decode CTAs co-located on the same SMs while the prefill is short):
     limited = (B > 0 and sum_i P_i <= 1536 and the unlimited ablation is
     off); slots = num_sms if limited (one prefill slot per SM: the SM's
-    other CTA, decode-home or a second prefill-home one, stays for decode;
-    measured on B200, a second prefill CTA adds only ~15% to an SM's prefill
-    throughput) else num_sms * k;
+    other CTA, decode-home or a second prefill-home one, stays for decode)
+    else num_sms * k;
     n0 = number of base items.  If prefill_splits == 1, or n0 == 0, or
     n0 >= slots: every item has S = 1 piece.  Otherwise W = sum of n over the
     base items, tau = max(8, ceil(W / slots)) and an item of n tiles gets

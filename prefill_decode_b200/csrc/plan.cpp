@@ -212,7 +212,7 @@ int pod_plan_build(const pod_attn_config* cfg, int num_sms, int32_t NP, const in
 
   // ---- prefill KV split: fill the prefill CTA slots when the base items leave some empty;
   // a short prefill (<= 1536 tokens) next to decode work counts one slot per SM (the SM's
-  // other CTA stays for decode; a second prefill CTA on an SM adds little throughput)
+  // other CTA stays for decode)
   {
     const bool limited = B > 0 && sumP <= kSplitLimitTokens && !(cfg->flags & POD_FLAG_PREFILL_SPLIT_UNLIMITED);
     const int64_t slots = limited ? (int64_t)num_sms : (int64_t)num_sms * k;
