@@ -238,6 +238,17 @@ def sample_sets(b, frac_den: int):
     return reqs, rows
 
 
+def single_launch(kw, info) -> bool:
+    """True when one step of a plan made with these keywords is one fused-kernel launch and nothing
+    else (no counter memset, no second kernel): its back-to-back step time is the kernel's time."""
+    import prefill_decode_b200 as pod
+    flags = kw.get("flags", 0)
+    if flags & (pod.POD_FLAG_SEQUENTIAL | pod.POD_FLAG_TRACE | pod.POD_FLAG_MERGE_KERNEL):
+        return False
+    two = flags & pod.POD_FLAG_TWO_STREAMS
+    return not (two and info.num_prefill_items > 0 and info.num_decode_items > 0)
+
+
 def fp8_alg_bytes(info, w) -> int:
     """Algorithmic bytes of a run whose decodes read e4m3 K/V (1 byte per element) and whose
     prefill requests read bf16 K/V: decode K/V + prefill K/V + Q + O."""
@@ -343,24 +354,30 @@ def run_sweep(args):
             torch.cuda.synchronize()
             est_s = e0.elapsed_time(e1) / 5e3
             steps = int(min(4000, max(args.steps, 0.4 / max(est_s, 1e-6))))
-            ev = [(pod.Event(), pod.Event()) for _ in range(steps)]
             t_w0 = time.time()
             e0.record(stream)
             for i in range(steps):
-                pl.set_events(ev[i][0].handle, ev[i][1].handle)
                 run()
             e1.record(stream)
             torch.cuda.synchronize()
             t_w1 = time.time()
+            step_us = e0.elapsed_time(e1) * 1e3 / steps
+            # then the same steps with events around each launch (kernel time with its launch latency)
+            ev = [(pod.Event(), pod.Event()) for _ in range(steps)]
+            for i in range(steps):
+                pl.set_events(ev[i][0].handle, ev[i][1].handle)
+                run()
+            torch.cuda.synchronize()
             pl.set_events(None, None)
             info = pl.info
-            step_us = e0.elapsed_time(e1) * 1e3 / steps
-            kern_us = float(np.mean([a.elapsed_ms(c) for a, c in ev])) * 1e3
+            kern_iso_us = float(np.mean([a.elapsed_ms(c) for a, c in ev])) * 1e3
+            kern_us = step_us if single_launch(kw, info) else kern_iso_us
             alg_bytes = fp8_alg_bytes(info, w) if use8 else info.kv_bytes + info.qo_bytes
             t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6
             t_tc = info.prefill_flops / (peaks["bf16_tflops"] * 1e12) * 1e6
             ck = sampler.summary(t_w0, t_w1)
-            res[mode] = {"steps": steps, "step_us": step_us, "kernel_us": kern_us, "roofline_us": max(t_hbm, t_tc),
+            res[mode] = {"steps": steps, "step_us": step_us, "kernel_us": kern_us, "kernel_us_isolated": kern_iso_us,
+                         "roofline_us": max(t_hbm, t_tc),
                          "frac_step": max(t_hbm, t_tc) / step_us, "frac_kernel": max(t_hbm, t_tc) / kern_us,
                          "bound": "hbm" if t_hbm >= t_tc else "tensor", "algorithmic_bytes": int(alg_bytes),
                          "hbm_GBps": alg_bytes / (kern_us * 1e-6) / 1e9,
@@ -443,7 +460,10 @@ def main():
         torch.cuda.synchronize(dev)
 
     def timed_loop(plan, wsp, K, per_step_events):
-        evs = [(pod.Event(), pod.Event()) for _ in range(K)] if per_step_events else []
+        # K steps back to back, events only at the two ends (an event between two launches would
+        # keep the fused kernel's CTAs from being scheduled while the previous one finishes);
+        # then, with per_step_events, K more steps with events around each launch for the
+        # kernel-only time
         for _ in range(args.warmup):
             db.run(pod, plan, wsp, stream=stream)
         barrier()
@@ -452,15 +472,20 @@ def main():
         t_wall0 = time.time()
         e0.record(stream)
         for i in range(K):
-            if per_step_events:
-                plan.set_events(evs[i][0].handle, evs[i][1].handle)
             db.run(pod, plan, wsp, stream=stream)
         e1.record(stream)
         barrier()
         t_wall1 = time.time()
-        plan.set_events(None, None)
         total_ms = e0.elapsed_time(e1)
-        kern = [a.elapsed_ms(c) for a, c in evs] if per_step_events else []
+        kern = []
+        if per_step_events:
+            evs = [(pod.Event(), pod.Event()) for _ in range(K)]
+            for i in range(K):
+                plan.set_events(evs[i][0].handle, evs[i][1].handle)
+                db.run(pod, plan, wsp, stream=stream)
+            plan.set_events(None, None)
+            torch.cuda.synchronize()
+            kern = [a.elapsed_ms(c) for a, c in evs]
         return total_ms, kern, (t_wall0, t_wall1)
 
     def max_over_ranks(x: float) -> float:
@@ -492,8 +517,10 @@ def main():
         pl_a.upload(ws_a, stream)
         # timed exactly like the fused arm (the same per-step events), so the step times compare directly
         a_ms, a_kern, _ = timed_loop(pl_a, ws_a, k_abl, True)
+        a_iso = float(np.mean(a_kern)) * 1e3
         ablations[name] = {"step_us": max_over_ranks(a_ms * 1e3 / k_abl),
-                           "kernels_us": max_over_ranks(float(np.mean(a_kern)) * 1e3),
+                           "kernels_us": max_over_ranks(a_ms * 1e3 / k_abl if single_launch(kw, pl_a.info) else a_iso),
+                           "kernels_us_isolated": max_over_ranks(a_iso),
                            "error_word": db.error_word(pl_a, ws_a)}
         del ws_a
     # the decode requests on an e4m3 copy of the cache (pod_attn_run_fp8kv), same plan and timing
@@ -547,7 +574,11 @@ def main():
     err_word = db.error_word(fused, ws)
 
     us = max_over_ranks(total_ms * 1e3 / args.steps)
-    kern_us = max_over_ranks(float(np.mean(kern_ms)) * 1e3)
+    # a step is one launch of the fused kernel and nothing else on the stream, so the timed region's
+    # average per step is the kernel's average launch duration (back to back, the gaps between
+    # launches included); the events around each launch give the time of one launch in isolation
+    kern_us = us
+    kern_iso_us = max_over_ranks(float(np.mean(kern_ms)) * 1e3)
     seq_us = max_over_ranks(seq_ms * 1e3 / max(50, args.steps // 4))
     seq_kern_us = max_over_ranks(float(np.mean(seq_kern)) * 1e3)
 
@@ -644,7 +675,11 @@ def main():
                      "achieved": achieved,
                      "peak": peak, "unit": unit, "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": traffic, "algorithmic_bytes": int(alg_bytes),
-                     "algorithmic_flops_prefill": int(info.prefill_flops), "kernel_us": kern_us},
+                     "algorithmic_flops_prefill": int(info.prefill_flops), "kernel_us": kern_us,
+                     "kernel_us_isolated": kern_iso_us,
+                     "kernel_us_note": "kernel_us = the timed region's events / steps (one launch per step, "
+                                       "back to back); kernel_us_isolated = mean of events recorded around "
+                                       "each launch in a second loop (launch latency exposed)"},
         "sequential_us": seq_us, "sequential_kernels_us": seq_kern_us, "speedup_vs_sequential": seq_us / us,
         "ablations": dict(ablations, fused_step_us=us,
                           note="two_streams = prefill-only and decode-only kernels on concurrent streams; "
@@ -655,8 +690,8 @@ def main():
                                "co-located-decode limit for <= 1536 prefill tokens off); prefill_split_never = "
                                "no prefill KV split"),
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
-        "launches_note": "per step: one pod_attn_kernel launch (split-KV rows merged inside it) after one "
-                         "cudaMemsetAsync of the workspace counters",
+        "launches_note": "per step: one pod_attn_kernel launch (split-KV rows merged inside it; its last CTA "
+                         "returns the workspace counters to zero, so no memset between steps)",
         "plan": {"prefill_items": info.num_prefill_items, "decode_items": info.num_decode_items,
                  "merge_items": info.num_merge_items, "chunk_pages": info.chunk_pages,
                  "ctas_per_sm": info.ctas_per_sm, "ratio": [info.ratio_prefill, info.ratio_decode],

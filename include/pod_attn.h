@@ -42,8 +42,10 @@
  * nothing aborts or throws across the ABI.  Device-side problems found while
  * the kernel runs (block id out of range, a bounded wait that expired, lengths
  * that disagree with the plan) are recorded as a negative code in the int32
- * error word at byte offset pod_attn_plan_info.error_offset of the workspace;
- * the offending access is skipped (a load reads zeros), so no fault is raised.
+ * error word at byte offset pod_attn_plan_info.error_offset of the workspace
+ * (the int32 after it holds the item or block involved); the offending access
+ * is skipped (a load reads zeros), so no fault is raised.  Once a run has
+ * completed in stream order, the word holds the first error of that run, or 0.
  */
 #ifndef POD_ATTN_H_
 #define POD_ATTN_H_
@@ -234,11 +236,17 @@ int pod_attn_plan_prefill_requests(const pod_attn_plan_t* plan, int32_t* out);
  * Errors: POD_ERR_INVALID_ARG, POD_ERR_WORKSPACE, POD_ERR_CUDA. */
 int pod_attn_upload(const pod_attn_plan_t* plan, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Enqueue one hybrid-batch attention on `stream`: reset the ticket, queue and
- * merge counters in the workspace, launch the persistent fused kernel (or, with
- * POD_FLAG_SEQUENTIAL in the plan's config, the prefill-only then decode-only
- * kernels; with POD_FLAG_TWO_STREAMS, the two on concurrent streams, the call
- * still completing in `stream` order).  Decode split-KV partials are merged by the warp that finishes a
+/* Enqueue one hybrid-batch attention on `stream`: launch the persistent fused
+ * kernel (or, with POD_FLAG_SEQUENTIAL in the plan's config, the prefill-only
+ * then decode-only kernels; with POD_FLAG_TWO_STREAMS, the two on concurrent
+ * streams, the call still completing in `stream` order).  The workspace's
+ * ticket, queue and merge counters must be zero when a launch starts:
+ * pod_attn_upload zeroes them, the fused kernel's last CTA returns them to zero
+ * (so consecutive runs on one workspace need no clearing in between), and the
+ * two-kernel and POD_FLAG_TRACE paths clear them with a memset first.  The
+ * fused kernel is launched with programmatic stream serialization: its CTAs may
+ * be scheduled while the previous kernel on `stream` finishes, and they wait for
+ * that kernel to complete before reading or writing global memory.  Decode split-KV partials are merged by the warp that finishes a
  * row's last split (a completion counter, no waiting), or, with POD_FLAG_MERGE_KERNEL,
  * by the LSE merge kernel launched afterwards; the KV pieces of a split prefill item
  * are always merged by the CTA that finishes the item's last piece.  Asynchronous.

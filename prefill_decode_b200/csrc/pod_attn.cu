@@ -87,6 +87,10 @@ struct alignas(64) PodParams {
   int32_t selftest_timeout; // 1: CTA 0 exercises the expired-wait path once
   int32_t partition_sms;   // > 0: roles by SM id instead of per-SM tickets (ablation)
   int32_t decode_warps;    // warps of a CTA that run decode items: 4, or 6 (the MMA and TMA warps too)
+  int32_t self_reset;      // 1 (a fused launch): errors go to the launch's own slot and the last CTA
+                           // out publishes them and returns every counter to zero
+  int32_t n_merge_cnt;     // ints of merge_cnt / pmerge_cnt (cleared by the last CTA after an error)
+  int32_t n_pmerge_cnt;
   float scale_log2;        // softmax scale * log2(e)
   const float* k_scale8;   // e4m3 caches: per kv head, dequantised value = scale * stored value
   const float* v_scale8;
@@ -162,8 +166,13 @@ static_assert(kAllWarps * Cfg<128>::kNSAll8 * Cfg<128>::kDecStage8 <= Cfg<128>::
                   Cfg<128>::kDecStage8 % 1024 == 0,
               "e4m3 decode rings exceed the shared-memory union or break the swizzle alignment");
 
+static_assert(kErrorInfo == kErrorWord + 1 && kRunErrorInfo == kRunError + 1, "error code and info are adjacent");
+
+// The first error of a launch wins.  A fused launch records into its own slot, which its last CTA
+// copies into the error word (so the word always tells about the last completed launch).
 __device__ __forceinline__ void record_error(const PodParams& p, int code, int info) {
-  if (atomicCAS(&p.counters[kErrorWord], 0, code) == 0) atomicExch(&p.counters[kErrorInfo], info);
+  const int w = p.self_reset ? kRunError : kErrorWord;
+  if (atomicCAS(&p.counters[w], 0, code) == 0) atomicExch(&p.counters[w + 1], info);
 }
 
 // Row of the K/V tensor maps holding page `blk`, kv head `kvh`; an
@@ -565,7 +574,10 @@ __device__ bool prefill_softmax(const PodParams& p, const PreItem& it, int item,
   __threadfence();
   __syncwarp();
   int last = 0;
-  if (lane == 0) last = atomicAdd(&p.pmerge_cnt[kWarpsPerCta * midx + warp], 1) == pm.y - 1;
+  if (lane == 0) {
+    last = atomicAdd(&p.pmerge_cnt[kWarpsPerCta * midx + warp], 1) == pm.y - 1;
+    if (last) p.pmerge_cnt[kWarpsPerCta * midx + warp] = 0;   // every piece has counted: ready for the next launch
+  }
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return true;
   __threadfence();
@@ -1143,7 +1155,10 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
         __threadfence();
         __syncwarp();
         int last = 0;
-        if (lane == 0) last = atomicAdd(&p.merge_cnt[midx], 1) == nsplit - 1;
+        if (lane == 0) {
+          last = atomicAdd(&p.merge_cnt[midx], 1) == nsplit - 1;
+          if (last) p.merge_cnt[midx] = 0;   // every split has counted: ready for the next launch
+        }
         last = __shfl_sync(0xffffffffu, last, 0);
         if (last) {
           __threadfence();
@@ -1168,7 +1183,10 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
   volatile int* sh_abort = reinterpret_cast<volatile int*>(ctrl + 3);
   const int tid = threadIdx.x, warp = tid >> 5;
   if (smem_u32(smem) & 1023u) {   // the swizzled tiles need 1024-byte alignment
-    if (tid == 0) record_error(p, POD_ERR_UNSUPPORTED, 1024);
+    if (tid == 0) {
+      griddep_wait();
+      record_error(p, POD_ERR_UNSUPPORTED, 1024);
+    }
     return;
   }
   if (tid == 0) {
@@ -1188,6 +1206,12 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
       tma_prefetch_desc(&p.tm_k8);
       tma_prefetch_desc(&p.tm_v8);
     }
+    // everything above touched only shared memory and the kernel parameters; the counters, the tables
+    // and the inputs may still be written by the grid this launch follows (programmatic dependent launch)
+    griddep_wait();
+    // and a dependent launch may be scheduled once every CTA of this grid got here (its CTAs take SMs
+    // only as this grid's CTAs leave them, and wait for this grid to complete before they start)
+    griddep_launch_dependents();
     int home = p.mode == kDecodeOnly ? kRoleDecode : kRolePrefill;
     if (p.mode == kFused && p.partition_sms > 0) {
       // ablation: whole SMs start on one role (the first partition_sms SM ids prefill-first)
@@ -1273,6 +1297,35 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
   if (p.use_tmem && warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  if (p.self_reset) {
+    // The last CTA out returns the launch's counters to zero for the next launch on this workspace (the
+    // warp that completes a merge has already reset that merge's count) and publishes the launch's
+    // first error, or none, in the error word.  No CTA of this launch touches the counters afterwards.
+    if (tid == 0) {
+      __threadfence();
+      ctrl[2] = atomicAdd(&p.counters[kExitCount], 1) == (int)gridDim.x - 1 ? 1u : 0u;
+    }
+    __syncthreads();
+    if (ctrl[2]) {
+      __threadfence();
+      volatile int32_t* c = p.counters;
+      const int err = c[kRunError];
+      for (int i = tid; i < kMaxSms; i += kThreads) c[kTicketBase + i] = 0;
+      if (err != 0) {   // an aborted launch can leave merges uncounted
+        for (int i = tid; i < p.n_merge_cnt; i += kThreads) p.merge_cnt[i] = 0;
+        for (int i = tid; i < p.n_pmerge_cnt; i += kThreads) p.pmerge_cnt[i] = 0;
+      }
+      if (tid == 0) {
+        c[kErrorInfo] = c[kRunErrorInfo];
+        c[kErrorWord] = err;
+        c[kRunError] = 0;
+        c[kRunErrorInfo] = 0;
+        c[kNextPrefill] = 0;
+        c[kNextDecode] = 0;
+        c[kExitCount] = 0;
+      }
+    }
   }
 }
 
@@ -1431,7 +1484,20 @@ int launch(const pod_attn_plan_t* pl, PodParams& prm, const MergeParams& mp, cud
   } else if (pl->n_pre > 0 || pl->n_dec > 0) {
     prm.mode = kFused;
     prm.use_tmem = pl->n_pre > 0 ? 1 : 0;
-    pod_attn_kernel<D, KV8><<<pl->grid, kThreads, smem, st>>>(prm);
+    // programmatic dependent launch: this grid's CTAs may be scheduled while the previous kernel on the
+    // stream finishes; they wait for it (griddep_wait) before touching global memory
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned)pl->grid);
+    lc.blockDim = dim3(kThreads);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    const cudaError_t le = cudaLaunchKernelEx(&lc, pod_attn_kernel<D, KV8>, prm);
+    if (le != cudaSuccess) return cuda_fail(le);
   }
   if (pl->ev_stop) cudaEventRecord(static_cast<cudaEvent_t>(pl->ev_stop), st);
   if (pl->n_merge > 0 && (pl->cfg.flags & POD_FLAG_MERGE_KERNEL))
@@ -1691,9 +1757,18 @@ int run_impl(const pod_attn_plan_t* pl, const void* q_prefill, const void* q_dec
   mp.Hq = Hq;
   mp.g = pl->g;
 
-  // counters (tickets, queue heads, error word, merge completions) start at zero every run
-  cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)pl->off_pre, st);
-  if (e != cudaSuccess) return cuda_fail(e);
+  prm.n_merge_cnt = pl->n_merge;
+  prm.n_pmerge_cnt = kWarpsPerCta * pl->n_pmerge;
+  // Counters (tickets, queue heads, error word, merge completions) are zero when a launch starts.  A
+  // fused launch leaves them at zero itself (its last CTA), so only the two-kernel paths, the traced
+  // path (its rescale count) and an empty batch (no launch, fresh error word) clear them here.
+  const uint32_t fl = pl->cfg.flags;
+  const bool two_kernels = (fl & POD_FLAG_SEQUENTIAL) || ((fl & POD_FLAG_TWO_STREAMS) && pl->n_pre > 0 && pl->n_dec > 0);
+  prm.self_reset = (pl->n_pre > 0 || pl->n_dec > 0) && !two_kernels && !(fl & POD_FLAG_TRACE) ? 1 : 0;
+  if (!prm.self_reset) {
+    const cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)pl->off_pre, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   if (f8 && has_dec) return D == 128 ? launch<128, true>(pl, prm, mp, st) : launch<64, true>(pl, prm, mp, st);
   return D == 128 ? launch<128, false>(pl, prm, mp, st) : launch<64, false>(pl, prm, mp, st);
 }

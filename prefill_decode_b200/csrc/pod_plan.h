@@ -17,7 +17,9 @@ constexpr int kMaxSms = 512;         // ticket slots (smid is folded modulo this
 constexpr int kCostRatio = 248;      // B200 tensor FLOP/s per HBM byte/s (1624.7e12 / 6539.5e9)
 
 // Workspace layout (bytes).  Counters first, then one completion counter per
-// decode merge item and per split prefill item (all zeroed every run); the
+// decode merge item and per split prefill item (zero whenever a launch starts:
+// pod_attn_upload zeroes them, a two-kernel or traced run zeroes them before
+// its launches, and a fused launch leaves them at zero when it ends); the
 // tables follow in the order prefill items | decode items | merge items |
 // prefill requests | prefill merge items; then the decode split partials
 // (O [n, g, d] and LSE [n, g], fp32) and the prefill piece partials
@@ -29,6 +31,9 @@ constexpr int kNextDecode = 513;     // int32
 constexpr int kErrorWord = 514;      // int32 (first error code recorded)
 constexpr int kErrorInfo = 515;      // int32 (item or block that caused it)
 constexpr int kRescaleCount = 516;   // int32: prefill softmax warps that rescaled O (counted with POD_FLAG_TRACE)
+constexpr int kExitCount = 517;      // int32: CTAs of a fused launch that have finished
+constexpr int kRunError = 518;       // int32: first error code of the fused launch in flight
+constexpr int kRunErrorInfo = 519;   // int32: item or block that caused it
 constexpr int kPrefillItemInts = 8;  // q0 (within the request), q_head, kv_end, prefill request,
                                      // first and end key tile (64 keys each), partial (-1 = unsplit), merge
 constexpr int kPrefillMergeInts = 4; // first partial, pieces, 0, 0

@@ -203,3 +203,59 @@ def test_split_prefill_trace_and_bad_block(env):
     assert np.isfinite(op).all()
     rd = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, 2)
     assert _close(od, rd)
+
+
+@pytest.mark.parametrize("name", ["decode_splits", "prefill_pieces"])
+def test_back_to_back_runs_reuse_the_workspace(env, name):
+    """A fused launch leaves its counters at zero (last CTA out; merge counts by the warp that
+    completes the merge), so repeated runs on one uploaded workspace stay correct without any
+    clearing in between."""
+    torch, pod = env
+    w = W if name == "decode_splits" else synth.custom("robust_split", 8, 2, 128, 256, 2000, [300, 1200], 34)
+    b = synth.make_batch(w)
+    db = DeviceBatch(torch, b)
+    pl = db.plan(pod)
+    assert pl.info.num_merge_items > 0
+    if name == "prefill_pieces":
+        assert pl.info.num_prefill_partials > 0
+    ws = db.workspace(pl)
+    pl.upload(ws)
+    rp = A.attend_prefill(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_ctx, b.scale, 2)
+    rd = A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, 2)
+    for _ in range(4):
+        db.o_pre.fill_(float("nan"))
+        db.o_dec.fill_(float("nan"))
+        db.run(pod, pl, ws)
+        torch.cuda.synchronize()
+        assert db.error_word(pl, ws) == 0
+        assert int(torch.count_nonzero(ws[:4096]).item()) == 0, "counters left non-zero"
+        op, od = db.outputs()
+        assert _close(op, rp) and _close(od, rd)
+
+
+def test_error_word_tells_about_the_last_run_only(env):
+    """A run that records an error publishes it; the next run on the same workspace, with the
+    block table repaired and no upload in between, reports 0 and is correct."""
+    torch, pod = env
+    b = synth.make_batch(W)
+    db = DeviceBatch(torch, b)
+    good = db.bt
+    bt = b.block_table.copy()
+    bt[3, 5] = 10 ** 6                  # decode request 2 (1500 tokens), page 5
+    pl = db.plan(pod)
+    ws = db.workspace(pl)
+    pl.upload(ws)
+    db.bt = torch.from_numpy(bt).cuda()
+    db.run(pod, pl, ws)
+    torch.cuda.synchronize()
+    assert db.error_word(pl, ws) == pod.POD_ERR_BOUNDS
+    off = pl.info.error_offset
+    assert int(ws[off + 4:off + 8].view(torch.int32).item()) == 10 ** 6
+    db.bt = good
+    db.run(pod, pl, ws)
+    torch.cuda.synchronize()
+    assert db.error_word(pl, ws) == 0
+    assert int(ws[off + 4:off + 8].view(torch.int32).item()) == 0
+    op, od = db.outputs()
+    assert _close(op, A.attend_prefill(b.q_prefill, b.k_pool, b.v_pool, b.block_table, b.prefill_ctx, b.scale, 2))
+    assert _close(od, A.attend_decode(b.q_decode, b.k_pool, b.v_pool, b.block_table, b.kv_lens, b.scale, 2))
