@@ -89,6 +89,7 @@ struct alignas(64) PodParams {
   int32_t decode_warps;    // warps of a CTA that run decode items: 4, or 6 (the MMA and TMA warps too)
   int32_t self_reset;      // 1 (a fused launch): errors go to the launch's own slot and the last CTA
                            // out publishes them and returns every counter to zero
+  int32_t n_ppart;         // prefill piece partials of the plan (0: no prefill item is split)
   int32_t n_merge_cnt;     // ints of merge_cnt / pmerge_cnt (cleared by the last CTA after an error)
   int32_t n_pmerge_cnt;
   float scale_log2;        // softmax scale * log2(e)
@@ -402,10 +403,9 @@ __device__ bool prefill_mma(const PodParams& p, const PreItem& it, uint8_t* smem
 // a lazily updated row max (O in TMEM is rescaled only when the max grows by
 // more than 2^8), write P_t as bf16 into shared-memory buffer t&1 in the
 // K-major 128B-swizzled layout.  Epilogue: O / l -> bf16 -> global, or, for
-// one KV piece of a split item, the piece's partial (O / l in fp32 and its
-// log-sum-exp) and then the log-sum-exp merge of all the item's pieces, done
-// for each warp's 32 rows by the warp that finishes those rows' last piece
-// (a completion counter per item and softmax warp: no warp waits on another).
+// one KV piece of a split item, the piece's partial rows (O / l in fp32) into
+// shared memory and their log-sum-exps into the workspace; the CTA finishes
+// the piece after the item's barrier (prefill_piece_end).
 template <int D>
 __device__ bool prefill_softmax(const PodParams& p, const PreItem& it, int item, uint8_t* smem, uint64_t* bars,
                                 uint32_t tmem, uint32_t t0, uint32_t nq) {
@@ -532,7 +532,7 @@ __device__ bool prefill_softmax(const PodParams& p, const PreItem& it, int item,
   __nv_bfloat16* orow = p.o_pre + ((size_t)(q_first + q) * p.Hq + qh) * D;
   // the piece fields are read again here rather than kept live through the tile loop
   const int4 piece = ld_nc_v4(&p.pre_items[2 * item + 1]);   // j0, j1, partial, merge
-  const int part = piece.z, midx = piece.w;
+  const int part = piece.z;
   if (part < 0) {
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
@@ -554,103 +554,23 @@ __device__ bool prefill_softmax(const PodParams& p, const PreItem& it, int item,
     }
     return true;
   }
-  // one KV piece of a split item: write this piece's partial row
-  float* prow_o = p.ppart_o + ((size_t)part * kBM + row) * D;
+  // One KV piece of a split item: each thread's row (O / l, fp32) goes to shared memory (the K ring, free
+  // once the item's last P.V MMA finished), row-major as the workspace holds it, and the row's log-sum-exp
+  // (log2 domain) to the workspace; after the item's barrier the CTA sends the tile out in one bulk copy
+  // and merges it if it was the last piece (prefill_piece_end).
+  float4* stg = reinterpret_cast<float4*>(smem + Cfg<D>::kOffK) + row * (D / 4);
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
     float o[32];
     tmem_ld32(tmem + t_lane + kTmemO + c * 32, o);
     tmem_wait_ld();
-    if (q < P) {
-      float4* dst = reinterpret_cast<float4*>(prow_o + c * 32);
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        dst[k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv, o[4 * k + 3] * inv);
-    }
+    for (int k = 0; k < 8; ++k)
+      stg[c * 8 + k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv, o[4 * k + 3] * inv);
   }
   if (q < P) p.ppart_lse[(size_t)part * kBM + row] = m + __log2f(l);
-  // the warp that finishes its rows' last piece merges them (no waiting on other warps or CTAs)
-  const int4 pm = __ldg(&p.pmerge_items[midx]);   // first partial, pieces
-  __threadfence();
-  __syncwarp();
-  int last = 0;
-  if (lane == 0) {
-    last = atomicAdd(&p.pmerge_cnt[kWarpsPerCta * midx + warp], 1) == pm.y - 1;
-    if (last) p.pmerge_cnt[kWarpsPerCta * midx + warp] = 0;   // every piece has counted: ready for the next launch
-  }
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last) return true;
-  __threadfence();
-  // O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s (log2 domain), over the warp's 32
-  // rows; the other pieces' partials were written by other CTAs of this launch: read them through L2.
-  // Each thread first turns its row's log-sum-exps into normalised weights (one batch of loads) and parks
-  // them in this warp's part of the P buffers (free: every P.V MMA of the item has finished); then it reads
-  // its row's partials two pieces per batch of loads, so a row costs about 1 + (d/32) * pieces/2 round trips
-  // (the epilogue of a split item took up to 30 us when every load waited for the one before).
-  const int first = pm.x, S = pm.y;
-  const int row0 = warp * 32;
-  float* wtab = reinterpret_cast<float*>(smem + Cfg<D>::kOffP) + warp * (kMaxPrefillPieces * 32);
-  {
-    // the (at most 16) log-sum-exps of lane's row in one batch of loads, then max, weights, sum
-    const float* lse = p.ppart_lse + (size_t)first * kBM + row0 + lane;
-    float M = -INFINITY;
-#pragma unroll
-    for (int sp = 0; sp < kMaxPrefillPieces; ++sp) {
-      if (sp < S) {
-        const float x = __ldcg(lse + (size_t)sp * kBM);
-        wtab[sp * 32 + lane] = x;
-        M = fmaxf(M, x);
-      }
-    }
-    float den = 0.f;
-#pragma unroll 1
-    for (int sp = 0; sp < S; ++sp) {
-      const float e = ex2(wtab[sp * 32 + lane] - M);
-      wtab[sp * 32 + lane] = e;
-      den += e;
-    }
-    const float dinv = 1.f / den;   // rows past the chunk (never written) give garbage weights, never used
-#pragma unroll 1
-    for (int sp = 0; sp < S; ++sp) wtab[sp * 32 + lane] *= dinv;
-  }
-  __syncwarp();
-  if (q >= P) return true;
-#pragma unroll 1
-  for (int c = 0; c < D / 32; ++c) {
-    float acc[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) acc[k] = 0.f;
-#pragma unroll 1
-    for (int sp = 0; sp < S; sp += 2) {
-      const int sp1 = sp + 1 < S ? sp + 1 : sp;   // a valid address either way; its weight is 0 then
-      const float wa = wtab[sp * 32 + lane], wb = sp + 1 < S ? wtab[sp1 * 32 + lane] : 0.f;
-      const float4* pa = reinterpret_cast<const float4*>(p.ppart_o + ((size_t)(first + sp) * kBM + row) * D + c * 32);
-      const float4* pb = reinterpret_cast<const float4*>(p.ppart_o + ((size_t)(first + sp1) * kBM + row) * D + c * 32);
-      float4 va[8], vb[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        va[k] = __ldcg(pa + k);
-        vb[k] = __ldcg(pb + k);
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        acc[4 * k] += wa * va[k].x + wb * vb[k].x;
-        acc[4 * k + 1] += wa * va[k].y + wb * vb[k].y;
-        acc[4 * k + 2] += wa * va[k].z + wb * vb[k].z;
-        acc[4 * k + 3] += wa * va[k].w + wb * vb[k].w;
-      }
-    }
-    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint4 v;
-      v.x = pack_bf16(acc[k * 8 + 0], acc[k * 8 + 1]);
-      v.y = pack_bf16(acc[k * 8 + 2], acc[k * 8 + 3]);
-      v.z = pack_bf16(acc[k * 8 + 4], acc[k * 8 + 5]);
-      v.w = pack_bf16(acc[k * 8 + 6], acc[k * 8 + 7]);
-      dst[k] = v;
-    }
-  }
+  fence_proxy_async_smem();   // the row is read by the bulk copy (async proxy) ...
+  __threadfence();            // ... and the log-sum-exp by other CTAs once the piece is counted
   return true;
 }
 
@@ -1169,6 +1089,115 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
   }
 }
 
+// The end of one KV piece of a split prefill item, by the whole CTA after the item's barrier (the
+// softmax threads have put the tile's 128 partial rows, O / l in fp32, row-major into the K ring and
+// their log-sum-exps into the workspace).  One thread sends the tile out in one bulk copy (the rows are
+// contiguous there as here) and counts the piece; the CTA that counts the item's last piece merges the
+// pieces: O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s (log2 domain).  Each of
+// threads 0..127 turns its row's log-sum-exps into normalised weights (in the P buffers, free as well);
+// then the six warps walk the rows with lanes along d, this piece's partial from shared memory and every
+// other piece's with one coalesced load per row (written by other CTAs of this launch: read through L2),
+// eight rows per lane in flight, and write the bf16 result as whole rows.  No CTA waits for another.
+template <int D>
+__device__ void prefill_piece_end(const PodParams& p, int item, uint8_t* smem, volatile uint32_t* flag) {
+  constexpr int kF4 = D / 4;            // float4 per row
+  constexpr int kRowsPer = 32 / kF4;    // rows per warp-wide access (1 at d = 128, 2 at d = 64)
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (p.n_ppart == 0) return;
+  // the piece fields are read again rather than kept live through the item
+  const int4 pc = ld_nc_v4(&p.pre_items[2 * item + 1]);   // j0, j1, partial, merge
+  const int part = pc.z, midx = pc.w;
+  if (part < 0) return;
+  const float4* stg = reinterpret_cast<const float4*>(smem + Cfg<D>::kOffK);
+  if (tid == 0) {
+    bulk_store_s2g(p.ppart_o + (size_t)part * kBM * D, stg, (uint32_t)(kBM * D * 4));
+    bulk_commit();
+    bulk_wait_all();              // the rows are in global memory (and the K ring may be reused) ...
+    fence_proxy_async_global();   // ... ordered before the count
+    __threadfence();
+    const int4 pm = ld_nc_v4(&p.pmerge_items[midx]);   // first partial, pieces
+    const bool last = atomicAdd(&p.pmerge_cnt[kWarpsPerCta * midx], 1) == pm.y - 1;
+    if (last) p.pmerge_cnt[kWarpsPerCta * midx] = 0;   // every piece has counted: ready for the next launch
+    *flag = last ? 1u : 0u;
+  }
+  __syncthreads();
+  if (*flag == 0u) return;
+  __threadfence();
+  const int4 pm = ld_nc_v4(&p.pmerge_items[midx]);
+  const int first = pm.x, S = pm.y, own = part - first;
+  const int4 ia = ld_nc_v4(&p.pre_items[2 * item]);      // q0, q head, kv_end, request
+  const int4 rq = __ldg(&p.pre_reqs[ia.w]);               // first row in q_pre / o_pre, P, C
+  const int rows_left = rq.y - ia.x;                      // tile rows r < rows_left are inside the chunk
+  float* wtab = reinterpret_cast<float*>(smem + Cfg<D>::kOffP);   // [piece][128 rows]
+  if (tid < kBM) {
+    const float* lse = p.ppart_lse + (size_t)first * kBM + tid;
+    float M = -INFINITY;
+#pragma unroll 4
+    for (int sp = 0; sp < S; ++sp) {
+      const float x = __ldcg(lse + (size_t)sp * kBM);
+      wtab[sp * kBM + tid] = x;
+      M = fmaxf(M, x);
+    }
+    float den = 0.f;
+    for (int sp = 0; sp < S; ++sp) {
+      const float e = ex2(wtab[sp * kBM + tid] - M);
+      wtab[sp * kBM + tid] = e;
+      den += e;
+    }
+    const float dinv = 1.f / den;   // rows past the chunk (never written) give garbage weights, never used
+    for (int sp = 0; sp < S; ++sp) wtab[sp * kBM + tid] *= dinv;
+  }
+  __syncthreads();
+  constexpr int kBatch = 8;                       // rows per lane in flight
+  constexpr int kSteps = kBM / kRowsPer;          // warp-wide row steps of the tile
+  const int sub = lane / kF4, f4 = lane % kF4;
+  const float4* part0 = reinterpret_cast<const float4*>(p.ppart_o) + ((size_t)first * kBM + sub) * kF4 + f4;
+  const size_t ostride = (size_t)p.Hq * D;
+  __nv_bfloat16* out0 = p.o_pre + ((size_t)(rq.x + ia.x + sub) * p.Hq + ia.y) * D + 4 * f4;
+  for (int s0 = warp; s0 < kSteps; s0 += kAllWarps * kBatch) {
+    // this warp's row steps s0, s0 + 6, ..., s0 + 6 (kBatch - 1): row r = step * kRowsPer + sub
+    float4 acc[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int st = s0 + u * kAllWarps;
+      const int r = (st < kSteps ? st : 0) * kRowsPer + sub;
+      const float w = wtab[own * kBM + r];
+      const float4 v = stg[r * kF4 + f4];
+      acc[u] = make_float4(w * v.x, w * v.y, w * v.z, w * v.w);
+    }
+    for (int sp = 0; sp < S; ++sp) {
+      if (sp == own) continue;
+      float4 va[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int st = s0 + u * kAllWarps;
+        va[u] = __ldcg(part0 + ((size_t)sp * kBM + (st < kSteps ? st : 0) * kRowsPer) * kF4);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int st = s0 + u * kAllWarps;
+        const float w = wtab[sp * kBM + (st < kSteps ? st : 0) * kRowsPer + sub];
+        acc[u].x += w * va[u].x;
+        acc[u].y += w * va[u].y;
+        acc[u].z += w * va[u].z;
+        acc[u].w += w * va[u].w;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int st = s0 + u * kAllWarps;
+      const int r = st * kRowsPer + sub;
+      if (st < kSteps && r < rows_left) {
+        uint2 v;
+        v.x = pack_bf16(acc[u].x, acc[u].y);
+        v.y = pack_bf16(acc[u].z, acc[u].w);
+        *reinterpret_cast<uint2*>(out0 + (size_t)st * kRowsPer * ostride) = v;
+      }
+    }
+  }
+  fence_proxy_async_smem();   // the next item's TMA loads reuse the K ring and the P buffers
+}
+
 // --------------------------------------------------------- persistent kernel
 // Grid = SMs x CTAs/SM.  Each CTA takes one ticket from its SM's counter; the
 // ticket fixes its home role (prefill iff t mod (p+d) < p).  The CTA drains
@@ -1283,6 +1312,7 @@ __global__ void __launch_bounds__(kThreads, 2) pod_attn_kernel(const __grid_cons
           __syncthreads();
           break;
         }
+        prefill_piece_end<D>(p, item, smem, ctrl + 4);
         tiles_done += (uint32_t)(it.j1 - it.j0);
         items_done += 1;
       }
@@ -1757,6 +1787,7 @@ int run_impl(const pod_attn_plan_t* pl, const void* q_prefill, const void* q_dec
   mp.Hq = Hq;
   mp.g = pl->g;
 
+  prm.n_ppart = pl->n_ppart;
   prm.n_merge_cnt = pl->n_merge;
   prm.n_pmerge_cnt = kWarpsPerCta * pl->n_pmerge;
   // Counters (tickets, queue heads, error word, merge completions) are zero when a launch starts.  A
