@@ -181,7 +181,7 @@ def test_planted_non_minimal_split_is_caught():
     check_plan(late, w.num_q_heads, w.num_kv_heads, 0, 0, lens, minc=pl.chunk_pages + 1)
     assert late.chunk_pages == pl.chunk_pages + 1
     with pytest.raises(AssertionError):
-        check_split_minimal(late, w.num_kv_heads, lens)   # judged by the default minimum of 16 pages
+        check_split_minimal(late, w.num_kv_heads, lens)   # checked against the default minimum of 16 pages
 
 
 @pytest.mark.parametrize("w", CONFIGS, ids=lambda w: w.name)
