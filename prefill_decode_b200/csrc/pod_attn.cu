@@ -554,8 +554,8 @@ __device__ bool prefill_softmax(const PodParams& p, const PreItem& it, int item,
     }
     return true;
   }
-  // One KV piece of a split item: each thread's row (O / l, fp32) goes to shared memory (the K ring, free
-  // once the item's last P.V MMA finished), row-major as the workspace holds it, and the row's log-sum-exp
+  // One KV piece of a split item: each thread's row (O / l, fp32) goes to shared memory (the K and V rings,
+  // free once the item's last P.V MMA finished), row-major as the workspace holds it, and the row's log-sum-exp
   // (log2 domain) to the workspace; after the item's barrier the CTA sends the tile out in one bulk copy
   // and merges it if it was the last piece (prefill_piece_end).
   float4* stg = reinterpret_cast<float4*>(smem + Cfg<D>::kOffK) + row * (D / 4);
@@ -1090,7 +1090,7 @@ __device__ bool decode_warp(const PodParams& p, uint8_t* ring, uint64_t* wbars, 
 }
 
 // The end of one KV piece of a split prefill item, by the whole CTA after the item's barrier (the
-// softmax threads have put the tile's 128 partial rows, O / l in fp32, row-major into the K ring and
+// softmax threads have put the tile's 128 partial rows, O / l in fp32, row-major into the K and V rings and
 // their log-sum-exps into the workspace).  One thread sends the tile out in one bulk copy (the rows are
 // contiguous there as here) and counts the piece; the CTA that counts the item's last piece merges the
 // pieces: O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s (log2 domain).  Each of
@@ -1112,7 +1112,7 @@ __device__ void prefill_piece_end(const PodParams& p, int item, uint8_t* smem, v
   if (tid == 0) {
     bulk_store_s2g(p.ppart_o + (size_t)part * kBM * D, stg, (uint32_t)(kBM * D * 4));
     bulk_commit();
-    bulk_wait_all();              // the rows are in global memory (and the K ring may be reused) ...
+    bulk_wait_all();              // the rows are in global memory (and the rings may be reused) ...
     fence_proxy_async_global();   // ... ordered before the count
     __threadfence();
     const int4 pm = ld_nc_v4(&p.pmerge_items[midx]);   // first partial, pieces
@@ -1195,7 +1195,7 @@ __device__ void prefill_piece_end(const PodParams& p, int item, uint8_t* smem, v
       }
     }
   }
-  fence_proxy_async_smem();   // the next item's TMA loads reuse the K ring and the P buffers
+  fence_proxy_async_smem();   // the next item's TMA loads reuse the rings and the P buffers
 }
 
 // --------------------------------------------------------- persistent kernel
