@@ -1,7 +1,8 @@
 """Host-side pieces of bench.py that need no GPU: the CPU-baseline sampling
 (which rows and requests, how sampled oracle time scales to the whole batch)
 for one and for several prefill requests, the device-code hash that keys the
-committed ncu traffic figure, and the plan digest replicas compare."""
+committed ncu traffic figure, the plan digest replicas compare, and which arms'
+step is a single kernel launch."""
 import numpy as np
 import pytest
 
@@ -70,3 +71,26 @@ def test_single_thread_oracle_figure_is_positive_and_scaled():
     v = bench.cpu_oracle_single_thread_us(b, reqs, rows)
     assert v > 0
     assert bench.blas_threads() >= 1
+
+
+def test_single_launch_names_the_arms_whose_step_is_one_kernel():
+    """The step of a plain fused plan is one launch (its kernel time is the back-to-back step time); the
+    two-kernel arms, the traced path and the separate merge kernel are not."""
+    import prefill_decode_b200 as pod
+
+    class Info:
+        def __init__(self, n_pre, n_dec):
+            self.num_prefill_items, self.num_decode_items = n_pre, n_dec
+
+    both = Info(4, 9)
+    assert bench.single_launch({}, both)
+    assert bench.single_launch(dict(ratio=(1, 0)), both)
+    assert bench.single_launch(dict(flags=pod.POD_FLAG_SM_PARTITION | pod.POD_FLAG_DECODE_FOUR_WARPS), both)
+    assert bench.single_launch(dict(flags=pod.POD_FLAG_PREFILL_SPLIT_UNLIMITED, max_prefill_splits=1), both)
+    assert not bench.single_launch(dict(flags=pod.POD_FLAG_SEQUENTIAL), both)
+    assert not bench.single_launch(dict(flags=pod.POD_FLAG_TWO_STREAMS), both)
+    assert not bench.single_launch(dict(flags=pod.POD_FLAG_TRACE), both)
+    assert not bench.single_launch(dict(flags=pod.POD_FLAG_MERGE_KERNEL), both)
+    # two streams with one side empty falls back to the fused launch
+    assert bench.single_launch(dict(flags=pod.POD_FLAG_TWO_STREAMS), Info(0, 9))
+    assert bench.single_launch(dict(flags=pod.POD_FLAG_TWO_STREAMS), Info(4, 0))
