@@ -229,10 +229,12 @@ int pod_attn_plan_prefill_merges(const pod_attn_plan_t* plan, int32_t* out);
  * Errors: POD_ERR_INVALID_ARG (null plan). */
 int pod_attn_plan_prefill_requests(const pod_attn_plan_t* plan, int32_t* out);
 
-/* Enqueue on `stream` (a cudaStream_t; NULL = legacy default stream) the copy
- * of the plan's work tables into `workspace` (device, >= workspace_bytes,
- * 256-byte aligned).  Call once per plan and workspace before pod_attn_run;
- * the host tables may be destroyed afterwards in stream order.
+/* Enqueue on `stream` (a cudaStream_t; NULL = legacy default stream) the
+ * zeroing of the workspace's counters and the copy of the plan's work tables
+ * into `workspace` (device, >= workspace_bytes, 256-byte aligned).  Call once
+ * per plan and workspace before pod_attn_run (runs on the same plan and
+ * workspace then need no further upload); the host tables may be destroyed
+ * afterwards in stream order.
  * Errors: POD_ERR_INVALID_ARG, POD_ERR_WORKSPACE, POD_ERR_CUDA. */
 int pod_attn_upload(const pod_attn_plan_t* plan, void* workspace, size_t workspace_bytes, void* stream);
 
